@@ -1,0 +1,165 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it and
+shares no code with it.  The arithmetic lives in ``attn_oracle.c`` (plain C,
+IEEE double); this module only builds it with gcc and marshals numpy arrays.
+
+What each function computes, and the passage it follows, is stated in the C
+file.  Pins (tests that tie the oracle to the pages and to mathematics rather
+than to itself) are in ``tests/test_oracle.py``.  Parity status of every
+function: pinned (closed forms, invariants, brute force, library special
+cases, finite differences).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+F64 = 0
+BF16 = 1
+
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, strict IEEE: no fast-math)."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra",
+           "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    if path is None and _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(path or build())
+    i64, dbl, vp, ip = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
+    lib.oracle_attention_forward.argtypes = [vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip, vp, vp]
+    lib.oracle_attention_forward_rows.argtypes = [vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip,
+                                                  vp, i64, vp, vp]
+    lib.oracle_attention_backward.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip,
+                                              vp, vp, vp]
+    lib.oracle_softmax_partial.argtypes = [vp, i64, vp, i64, vp, vp, vp]
+    lib.oracle_softmax_merge.argtypes = [dbl, dbl, vp, dbl, dbl, vp, i64, vp, vp, vp]
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ip]
+    for name in ("oracle_attention_forward", "oracle_attention_forward_rows",
+                 "oracle_attention_backward", "oracle_softmax_partial",
+                 "oracle_softmax_merge"):
+        getattr(lib, name).restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _as_input(x):
+    """Return (contiguous array, dtype code).  bf16 arrives as uint16 bits."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float64:
+        return x, F64
+    if x.dtype == np.uint16:
+        return x, BF16
+    raise TypeError(f"oracle inputs must be float64 or bf16 bits (uint16), got {x.dtype}")
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"{what} failed with code {rc}")
+
+
+def attention_forward(Q, K, V, scale: float, causal: bool, lib=None):
+    """O [B,H,N,d] and LSE [B,H,N] (float64) of softmax(Q K^T scale [+causal]) V."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv) = _as_input(Q), _as_input(K), _as_input(V)
+    assert dt == dk == dv and Q.shape == K.shape == V.shape and Q.ndim == 4
+    B, H, N, d = Q.shape
+    O = np.empty((B, H, N, d), np.float64)
+    LSE = np.empty((B, H, N), np.float64)
+    _check(lib.oracle_attention_forward(_ptr(Q), _ptr(K), _ptr(V), dt, B, H, N, d,
+                                        float(scale), int(bool(causal)), _ptr(O), _ptr(LSE)),
+           "oracle_attention_forward")
+    return O, LSE
+
+
+def attention_forward_rows(Q, K, V, scale: float, causal: bool, rows, lib=None):
+    """Rows of the forward: rows[k] = bh*N + i.  Returns O_rows [n,d], LSE_rows [n]."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv) = _as_input(Q), _as_input(K), _as_input(V)
+    assert dt == dk == dv and Q.shape == K.shape == V.shape and Q.ndim == 4
+    B, H, N, d = Q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    O = np.empty((rows.size, d), np.float64)
+    LSE = np.empty((rows.size,), np.float64)
+    _check(lib.oracle_attention_forward_rows(_ptr(Q), _ptr(K), _ptr(V), dt, B, H, N, d,
+                                             float(scale), int(bool(causal)), _ptr(rows),
+                                             rows.size, _ptr(O), _ptr(LSE)),
+           "oracle_attention_forward_rows")
+    return O, LSE
+
+
+def attention_backward(Q, K, V, dO, scale: float, causal: bool, lib=None):
+    """dQ, dK, dV [B,H,N,d] (float64): exact gradient of <O, dO>."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv), (dO, dd) = (_as_input(Q), _as_input(K), _as_input(V),
+                                           _as_input(dO))
+    assert dt == dk == dv == dd and Q.shape == K.shape == V.shape == dO.shape
+    B, H, N, d = Q.shape
+    dQ = np.empty((B, H, N, d), np.float64)
+    dK = np.empty_like(dQ)
+    dV = np.empty_like(dQ)
+    _check(lib.oracle_attention_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), dt, B, H, N, d,
+                                         float(scale), int(bool(causal)),
+                                         _ptr(dQ), _ptr(dK), _ptr(dV)),
+           "oracle_attention_backward")
+    return dQ, dK, dV
+
+
+def softmax_partial(s, Vblk, lib=None):
+    """(m, l, o) of one block of scores s [n] with value rows Vblk [n, d]."""
+    lib = lib or load()
+    s = np.ascontiguousarray(s, np.float64)
+    Vblk = np.ascontiguousarray(Vblk, np.float64)
+    d = Vblk.shape[1]
+    m, l = ctypes.c_double(), ctypes.c_double()
+    o = np.empty((d,), np.float64)
+    _check(lib.oracle_softmax_partial(_ptr(s), s.size, _ptr(Vblk), d, ctypes.byref(m),
+                                      ctypes.byref(l), _ptr(o)), "oracle_softmax_partial")
+    return m.value, l.value, o
+
+
+def softmax_merge(part_x, part_y, lib=None):
+    """Merge two (m, l, o) partials into the partial of the union of both blocks."""
+    lib = lib or load()
+    (mx, lx, ox), (my, ly, oy) = part_x, part_y
+    ox = np.ascontiguousarray(ox, np.float64)
+    oy = np.ascontiguousarray(oy, np.float64)
+    m, l = ctypes.c_double(), ctypes.c_double()
+    o = np.empty_like(ox)
+    _check(lib.oracle_softmax_merge(mx, lx, _ptr(ox), my, ly, _ptr(oy), ox.size,
+                                    ctypes.byref(m), ctypes.byref(l), _ptr(o)),
+           "oracle_softmax_merge")
+    return m.value, l.value, o
+
+
+def num_threads(lib=None) -> int:
+    return (lib or load()).oracle_num_threads()
+
+
+def set_num_threads(n: int, lib=None) -> None:
+    (lib or load()).oracle_set_num_threads(int(n))

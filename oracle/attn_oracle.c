@@ -1,0 +1,351 @@
+/*
+ * attn_oracle.c -- plain, slow, fp64 CPU oracle for exact scaled-dot-product
+ * attention and its gradient.
+ *
+ * THIS IS TEST INFRASTRUCTURE.  Only the test-suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load it.  It shares no code, header,
+ * table or helper with the CUDA library; it computes every result from the
+ * definitions below, in IEEE double precision, with no tiling, no online
+ * softmax and no reordering beyond what the definitions state.
+ *
+ * Sources (the web pages this method is described on):
+ *   [STD]   unite.ai, "Flash Attention: Revolutionizing Transformer
+ *           Efficiency" -- the standard-attention definition
+ *           softmax(Q K^T / sqrt(d_k)) V, with the (batch, seq, seq) score
+ *           tensor materialised.
+ *   [SAFE]  same page, "The math behind Flash Attention", item 1: the softmax
+ *           of x is exp(x - m) / sum exp(x - m), m = max(x).
+ *   [MERGE] same page, same section, item 2: two partial softmaxes are
+ *           combined by rescaling each with exp(m_x - m), exp(m_y - m),
+ *           m = max(m_x, m_y).  The printed formula is garbled; the reading
+ *           implemented in oracle_softmax_merge is stated there.
+ *   [RECOMP] same page, "Enter Flash Attention", idea 2: the backward pass
+ *           recomputes attention instead of storing it.  The pages print no
+ *           backward formulas; oracle_attention_backward is the exact
+ *           gradient of [STD].
+ *   [CAUSAL] downcodes.com, "triton transformer", usage section: the
+ *           `causal = True` (autoregressive) flag.  Reading: square,
+ *           top-left aligned -- query i sees keys j <= i.
+ *
+ * Readings where the pages are silent:
+ *   - scale is an explicit argument (the pages fix 1/sqrt(d));
+ *   - LSE_i = ln sum_j exp(s_ij) in natural-log units of the SCALED scores;
+ *   - masked scores are -inf and contribute exp(-inf) = 0.
+ *
+ * Inputs are either IEEE doubles (dtype ORACLE_F64) or bfloat16 bit patterns
+ * (dtype ORACLE_BF16, widened exactly to double on load).  Layout of every
+ * tensor: contiguous [B, H, N, d] (d fastest); LSE is [B, H, N].
+ *
+ * Every function returns 0 on success, -1 on a bad argument, -2 if memory
+ * could not be allocated.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_F64 0
+#define ORACLE_BF16 1
+
+/* Load element i of an input tensor as a double (bf16 widening is exact). */
+static double ld(const void *p, int64_t i, int dtype)
+{
+    if (dtype == ORACLE_F64)
+        return ((const double *)p)[i];
+    uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+static int bad_shape(int64_t B, int64_t H, int64_t N, int64_t d, int dtype)
+{
+    return B < 1 || H < 1 || N < 1 || d < 1 ||
+           (dtype != ORACLE_F64 && dtype != ORACLE_BF16);
+}
+
+/*
+ * One output row of [STD] for query i of head bh:
+ *   s_j   = scale * <q_i, k_j>           (s_j = -inf if causal and j > i)
+ *   m     = max_j s_j                    ([SAFE])
+ *   LSE_i = m + ln sum_j exp(s_j - m)
+ *   P_j   = exp(s_j - m) / sum_j exp(s_j - m)
+ *   O_i   = sum_j P_j v_j
+ * s is caller-provided scratch of N doubles.
+ */
+static void attention_row(const void *Q, const void *K, const void *V, int dtype,
+                          int64_t N, int64_t d, int64_t bh, int64_t i,
+                          double scale, int causal, double *s,
+                          double *o_row, double *lse)
+{
+    const int64_t base = bh * N * d;
+    for (int64_t j = 0; j < N; ++j) {
+        if (causal && j > i) {
+            s[j] = -INFINITY;
+            continue;
+        }
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+            acc += ld(Q, base + i * d + c, dtype) * ld(K, base + j * d + c, dtype);
+        s[j] = scale * acc;
+    }
+    double m = -INFINITY;
+    for (int64_t j = 0; j < N; ++j)
+        m = fmax(m, s[j]);
+    double sum = 0.0;
+    for (int64_t j = 0; j < N; ++j) {
+        s[j] = exp(s[j] - m); /* exp(-inf) = 0 for masked keys */
+        sum += s[j];
+    }
+    *lse = m + log(sum);
+    for (int64_t c = 0; c < d; ++c)
+        o_row[c] = 0.0;
+    for (int64_t j = 0; j < N; ++j) {
+        const double p = s[j] / sum;
+        if (p == 0.0)
+            continue;
+        for (int64_t c = 0; c < d; ++c)
+            o_row[c] += p * ld(V, base + j * d + c, dtype);
+    }
+}
+
+/* Full forward: O [B,H,N,d] and LSE [B,H,N], both double. */
+int oracle_attention_forward(const void *Q, const void *K, const void *V, int dtype,
+                             int64_t B, int64_t H, int64_t N, int64_t d,
+                             double scale, int causal, double *O, double *LSE)
+{
+    if (!Q || !K || !V || !O || !LSE || bad_shape(B, H, N, d, dtype))
+        return -1;
+    const int64_t rows = B * H * N;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc((size_t)N * sizeof(double));
+        if (!s) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < rows; ++r) {
+            if (!s)
+                continue;
+            const int64_t bh = r / N, i = r % N;
+            attention_row(Q, K, V, dtype, N, d, bh, i, scale, causal, s,
+                          O + r * d, LSE + r);
+        }
+        free(s);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Forward for a sample of rows only.  rows[k] = bh * N + i names query i of
+ * head bh; O_rows is [n_rows, d], LSE_rows is [n_rows].  Each output row of
+ * [STD] depends only on its own query and on all keys/values of its head, so
+ * a sampled row equals the same row of the full forward.
+ */
+int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, int dtype,
+                                  int64_t B, int64_t H, int64_t N, int64_t d,
+                                  double scale, int causal,
+                                  const int64_t *rows, int64_t n_rows,
+                                  double *O_rows, double *LSE_rows)
+{
+    if (!Q || !K || !V || !rows || !O_rows || !LSE_rows || n_rows < 0 ||
+        bad_shape(B, H, N, d, dtype))
+        return -1;
+    for (int64_t k = 0; k < n_rows; ++k)
+        if (rows[k] < 0 || rows[k] >= B * H * N)
+            return -1;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc((size_t)N * sizeof(double));
+        if (!s) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t k = 0; k < n_rows; ++k) {
+            if (!s)
+                continue;
+            const int64_t bh = rows[k] / N, i = rows[k] % N;
+            attention_row(Q, K, V, dtype, N, d, bh, i, scale, causal, s,
+                          O_rows + k * d, LSE_rows + k);
+        }
+        free(s);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Exact gradient of [STD] for upstream gradient dO, one head at a time,
+ * with the full N x N matrices P, dP and dS materialised ([RECOMP] says only
+ * that the fast path recomputes instead of storing; the oracle stores).
+ *   P_ij  = softmax_j(s_ij)                  (row i, masked keys give 0)
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = <dO_i, v_j>
+ *   D_i   = sum_j P_ij dP_ij
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale sum_j dS_ij k_j
+ *   dK_j  = scale sum_i dS_ij q_i
+ * Outputs dQ, dK, dV are double [B,H,N,d].
+ */
+int oracle_attention_backward(const void *Q, const void *K, const void *V, const void *dO,
+                              int dtype, int64_t B, int64_t H, int64_t N, int64_t d,
+                              double scale, int causal, double *dQ, double *dK, double *dV)
+{
+    if (!Q || !K || !V || !dO || !dQ || !dK || !dV || bad_shape(B, H, N, d, dtype))
+        return -1;
+    double *P = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
+    double *dS = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
+    if (!P || !dS) {
+        free(P);
+        free(dS);
+        return -2;
+    }
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t base = bh * N * d;
+        /* P row by row, exactly as the forward defines it. */
+#pragma omp parallel for schedule(dynamic, 8)
+        for (int64_t i = 0; i < N; ++i) {
+            double *s = P + i * N;
+            for (int64_t j = 0; j < N; ++j) {
+                if (causal && j > i) {
+                    s[j] = -INFINITY;
+                    continue;
+                }
+                double acc = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    acc += ld(Q, base + i * d + c, dtype) * ld(K, base + j * d + c, dtype);
+                s[j] = scale * acc;
+            }
+            double m = -INFINITY;
+            for (int64_t j = 0; j < N; ++j)
+                m = fmax(m, s[j]);
+            double sum = 0.0;
+            for (int64_t j = 0; j < N; ++j) {
+                s[j] = exp(s[j] - m);
+                sum += s[j];
+            }
+            for (int64_t j = 0; j < N; ++j)
+                s[j] /= sum;
+        }
+        /* dP, D and dS. */
+#pragma omp parallel for schedule(dynamic, 8)
+        for (int64_t i = 0; i < N; ++i) {
+            double *ds = dS + i * N;
+            for (int64_t j = 0; j < N; ++j) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    acc += ld(dO, base + i * d + c, dtype) * ld(V, base + j * d + c, dtype);
+                ds[j] = acc; /* dP_ij */
+            }
+            double D = 0.0;
+            for (int64_t j = 0; j < N; ++j)
+                D += P[i * N + j] * ds[j];
+            for (int64_t j = 0; j < N; ++j)
+                ds[j] = P[i * N + j] * (ds[j] - D);
+        }
+        /* dQ_i = scale sum_j dS_ij k_j */
+#pragma omp parallel for schedule(dynamic, 8)
+        for (int64_t i = 0; i < N; ++i) {
+            for (int64_t c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < N; ++j)
+                    acc += dS[i * N + j] * ld(K, base + j * d + c, dtype);
+                dQ[base + i * d + c] = scale * acc;
+            }
+        }
+        /* dK_j = scale sum_i dS_ij q_i ;  dV_j = sum_i P_ij dO_i */
+#pragma omp parallel for schedule(dynamic, 8)
+        for (int64_t j = 0; j < N; ++j) {
+            for (int64_t c = 0; c < d; ++c) {
+                double acc_k = 0.0, acc_v = 0.0;
+                for (int64_t i = 0; i < N; ++i) {
+                    acc_k += dS[i * N + j] * ld(Q, base + i * d + c, dtype);
+                    acc_v += P[i * N + j] * ld(dO, base + i * d + c, dtype);
+                }
+                dK[base + j * d + c] = scale * acc_k;
+                dV[base + j * d + c] = acc_v;
+            }
+        }
+    }
+    free(P);
+    free(dS);
+    return 0;
+}
+
+/*
+ * [SAFE] applied to one block of scores: for scores s[0..n) and value rows
+ * Vblk [n, d] (double), returns the block's max m, its sum
+ * l = sum exp(s - m), and the block-normalised output
+ * o = sum_j exp(s_j - m) v_j / l.  Used only to test [MERGE].
+ */
+int oracle_softmax_partial(const double *s, int64_t n, const double *Vblk, int64_t d,
+                           double *m, double *l, double *o)
+{
+    if (!s || !Vblk || !m || !l || !o || n < 1 || d < 1)
+        return -1;
+    double mx = -INFINITY;
+    for (int64_t j = 0; j < n; ++j)
+        mx = fmax(mx, s[j]);
+    double sum = 0.0;
+    for (int64_t j = 0; j < n; ++j)
+        sum += exp(s[j] - mx);
+    for (int64_t c = 0; c < d; ++c)
+        o[c] = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        const double w = exp(s[j] - mx) / sum;
+        for (int64_t c = 0; c < d; ++c)
+            o[c] += w * Vblk[j * d + c];
+    }
+    *m = mx;
+    *l = sum;
+    return 0;
+}
+
+/*
+ * [MERGE], read as: with m = max(m_x, m_y),
+ *   l = exp(m_x - m) l_x + exp(m_y - m) l_y
+ *   o = (exp(m_x - m) l_x o_x + exp(m_y - m) l_y o_y) / l
+ * where o_x, o_y are the block-normalised partial outputs.  The result is the
+ * softmax-weighted output over the union of both blocks.
+ */
+int oracle_softmax_merge(double m_x, double l_x, const double *o_x,
+                         double m_y, double l_y, const double *o_y, int64_t d,
+                         double *m, double *l, double *o)
+{
+    if (!o_x || !o_y || !m || !l || !o || d < 1)
+        return -1;
+    const double mm = fmax(m_x, m_y);
+    const double a = exp(m_x - mm) * l_x;
+    const double b = exp(m_y - mm) * l_y;
+    const double ll = a + b;
+    for (int64_t c = 0; c < d; ++c)
+        o[c] = (a * o_x[c] + b * o_y[c]) / ll;
+    *m = mm;
+    *l = ll;
+    return 0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
