@@ -1,0 +1,112 @@
+/*
+ * fa.h -- C ABI of libfa_sm100: exact IO-aware scaled-dot-product attention
+ * (FlashAttention-2 style) for NVIDIA B200 (sm_100a).
+ *
+ * The operation (unite.ai, "Flash Attention: Revolutionizing Transformer
+ * Efficiency", standard-attention definition; causal flag as in
+ * downcodes.com "triton transformer", usage section):
+ *
+ *     S   = scale * Q K^T,  S_ij = -inf where causal and j > i
+ *     O   = softmax_rows(S) V
+ *     LSE = log(sum_j exp(S_ij))            (natural log, scaled scores)
+ *
+ * computed in tiles with an online softmax so that S never reaches HBM
+ * (same page, "Flash Attention algorithm" and "math behind Flash
+ * Attention"); the backward recomputes S from LSE instead of storing it
+ * (same page, idea 2, "recomputation").
+ *
+ * Conventions shared by every entry point
+ *   - Layout: Q, K, V, O, dO, dQ, dK, dV are contiguous [B, H, N, d] bf16
+ *     (__nv_bfloat16, d fastest); LSE is contiguous [B, H, N] float32.
+ *   - All pointers are DEVICE pointers on the current CUDA device, 16-byte
+ *     aligned.  The caller allocates and owns every buffer; the library
+ *     allocates no device memory.
+ *   - d must be 64 or 128; B, H, N >= 1; B*H*N*d < 2^31; scale finite, > 0.
+ *   - causal != 0 selects the square, top-left aligned mask: query i attends
+ *     to keys j <= i.
+ *   - Work is enqueued on `stream` (0 = legacy default stream) and returns
+ *     without host synchronisation.  Outputs are fully overwritten.
+ *   - Errors: arguments are checked before any launch.  Invalid arguments
+ *     return FA_ERR_INVALID_ARG, unsupported shapes or devices
+ *     FA_ERR_UNSUPPORTED, launch failures FA_ERR_CUDA.  Nothing is thrown,
+ *     nothing exits.  Device-side waits are bounded; a wait that gives up
+ *     records a code in a per-device error word read by
+ *     fa_check_device_error (FA_ERR_TIMEOUT).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,
+    FA_ERR_UNSUPPORTED = 2,
+    FA_ERR_CUDA = 3,
+    FA_ERR_TIMEOUT = 4
+} fa_status;
+
+/*
+ * Forward pass.
+ *   Q, K, V : [B,H,N,d] bf16 inputs (read only)
+ *   O       : [B,H,N,d] bf16 output
+ *   LSE     : [B,H,N]   fp32 output, natural-log logsumexp of the scaled
+ *             scores per query row (needed by fa_backward)
+ * Numerics: bf16 operands, fp32 accumulation and softmax statistics; P is
+ * rounded to bf16 for the P.V product; O rounded to bf16 (nearest-even).
+ */
+fa_status fa_forward(const void *Q, const void *K, const void *V, void *O, float *LSE,
+                     int B, int H, int N, int d, float scale, int causal,
+                     cudaStream_t stream);
+
+/*
+ * Device workspace fa_backward needs, in bytes (0 on invalid shapes).  It holds
+ * D_i = <dO_i, O_i>, LSE in base-2 units and the fp32 dQ accumulator, each
+ * padded to a multiple of 128 rows per head.
+ */
+size_t fa_backward_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass: the exact gradient of <O, dO> with respect to Q, K and V,
+ * recomputing the scores from Q, K and the saved LSE (same page, idea 2).
+ *   Q, K, V, O, dO : [B,H,N,d] bf16 (read only); O and LSE from fa_forward
+ *   LSE            : [B,H,N] fp32 (read only)
+ *   dQ, dK, dV     : [B,H,N,d] bf16 outputs
+ *   workspace      : >= fa_backward_workspace_bytes(B,H,N,d) bytes of device
+ *                    memory, 16-byte aligned, owned by the caller, contents
+ *                    undefined on entry and exit; it must not be shared with
+ *                    another call that may run concurrently.
+ * dQ is accumulated in fp32 across key blocks with atomic reductions, so its
+ * last fp32 bits (and rarely one bf16 ulp) may vary from run to run; dK and
+ * dV are deterministic.
+ */
+fa_status fa_backward(const void *Q, const void *K, const void *V, const void *O,
+                      const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
+                      void *workspace, size_t workspace_bytes,
+                      int B, int H, int N, int d, float scale, int causal,
+                      cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word.  Returns FA_OK, FA_ERR_TIMEOUT if a kernel gave up at a bounded wait
+ * since the last check (its outputs are then undefined), or FA_ERR_CUDA.
+ * If site != NULL it receives the raw code (0 if none).
+ */
+fa_status fa_check_device_error(cudaStream_t stream, unsigned int *site);
+
+/* Static description of a status code. */
+const char *fa_status_str(fa_status status);
+
+/* Library ABI version (major * 100 + minor). */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

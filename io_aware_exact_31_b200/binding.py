@@ -1,0 +1,157 @@
+"""ctypes binding of libfa_sm100.so (argument marshalling only).
+
+PyTorch supplies device memory and the current stream; every step of the
+attention path runs in the library's CUDA kernels.  There is no fallback: if
+the library is missing or the device is not sm_100, calls raise ``FaError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+
+# Every entry point include/fa.h declares.
+EXPORTS = ("fa_forward", "fa_backward_workspace_bytes", "fa_backward", "fa_check_device_error",
+           "fa_status_str", "fa_version")
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} (status {status})")
+
+
+def load_library(path: str | None = None):
+    """Open the C-ABI library (once).  Raises FaError if it was not built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FaError(FA_ERR_UNSUPPORTED,
+                      f"{p} not found; build it with `python -m io_aware_exact_31_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_forward.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_forward.restype = i
+    lib.fa_backward_workspace_bytes.argtypes = [i, i, i, i]
+    lib.fa_backward_workspace_bytes.restype = sz
+    lib.fa_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+    lib.fa_backward.restype = i
+    lib.fa_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    lib.fa_check_device_error.restype = i
+    lib.fa_status_str.argtypes = [i]
+    lib.fa_status_str.restype = ctypes.c_char_p
+    lib.fa_version.restype = i
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    try:
+        return load_library().fa_status_str(status).decode()
+    except FaError:
+        return "library not loaded"
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_qkv(*ts):
+    shape = ts[0].shape
+    for t in ts:
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous bf16 CUDA tensors [B, H, N, d]")
+        if t.shape != shape or t.dim() != 4:
+            raise ValueError(f"shape mismatch: {tuple(t.shape)} vs {tuple(shape)}")
+    return shape
+
+
+def forward_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d, scale, causal, stream=0) -> int:
+    """fa_forward on raw device addresses; returns the status code."""
+    return load_library().fa_forward(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, N, d,
+                                     float(scale), int(bool(causal)), ctypes.c_void_p(stream))
+
+
+def backward_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa_backward_workspace_bytes(B, H, N, d))
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+            scale: float | None = None, out: torch.Tensor | None = None,
+            lse: torch.Tensor | None = None, stream=None):
+    """O, LSE = softmax(scale Q K^T [+causal]) V and its per-row logsumexp."""
+    B, H, N, d = _check_qkv(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check_qkv(q, o)
+    if l.dtype != torch.float32 or not l.is_contiguous() or tuple(l.shape) != (B, H, N):
+        raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
+    st = load_library().fa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   l.data_ptr(), B, H, N, d, scale, int(bool(causal)),
+                                   _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_forward")
+    return o, l
+
+
+def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
+             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, stream=None):
+    """dQ, dK, dV of <O, dO> (scores recomputed from the saved LSE)."""
+    B, H, N, d = _check_qkv(q, k, v, o, do)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    lib = load_library()
+    ws_bytes = int(lib.fa_backward_workspace_bytes(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib.fa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                         lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         B, H, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_backward")
+    return dq, dk, dv
+
+
+def check_device_error(stream=None) -> tuple[int, int]:
+    """Synchronise and read/clear the device error word: (status, raw site code)."""
+    site = ctypes.c_uint(0)
+    st = load_library().fa_check_device_error(_stream_handle(stream), ctypes.byref(site))
+    return st, site.value
+
+
+class _Attention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale):
+        o, lse = forward(q, k, v, causal=causal, scale=scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.causal, ctx.scale = causal, scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, o, do.contiguous(), lse, causal=ctx.causal,
+                              scale=ctx.scale)
+        return dq, dk, dv, None, None
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None):
+    """Differentiable exact attention (autograd wrapper over forward/backward)."""
+    return _Attention.apply(q, k, v, causal, scale)

@@ -1,0 +1,191 @@
+// fa_api.cu -- the C ABI (include/fa.h): argument validation, TMA descriptor
+// creation and kernel launch.  All arithmetic of the attention path runs in
+// the kernels of fa_fwd.cuh / fa_bwd.cuh.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+#include "tma_host.h"
+
+namespace fa {
+
+// Per-device error word written by bounded waits that gave up (0 = none).
+__device__ uint32_t g_err_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool checked = false;
+    bool supported = false;
+    uint32_t* err = nullptr;  // device address of g_err_word on this device
+    bool fwd_attr[2] = {false, false};
+    bool bwd_attr[2] = {false, false};
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Returns the state of the current device, or null if it is not a usable sm_100 part.
+DeviceState* current_device(fa_status* st) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *st = FA_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& s = g_dev[dev];
+    if (!s.checked) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            *st = FA_ERR_CUDA;
+            return nullptr;
+        }
+        s.supported = (major == 10 && minor == 0);
+        if (s.supported) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) {
+                *st = FA_ERR_CUDA;
+                return nullptr;
+            }
+            s.err = static_cast<uint32_t*>(p);
+        }
+        s.checked = true;
+    }
+    if (!s.supported) {
+        *st = FA_ERR_UNSUPPORTED;
+        return nullptr;
+    }
+    *st = FA_OK;
+    return &s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_shape(int B, int H, int N, int d, float scale) {
+    if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    const int64_t total = static_cast<int64_t>(B) * H * N * d;
+    if (total >= (int64_t(1) << 31) || static_cast<int64_t>(B) * H > 65535LL * 65535LL)
+        return FA_ERR_UNSUPPORTED;
+    if (H > 65535 || B > 65535) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+template <int D>
+fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const void* V, void* O,
+                         float* LSE, int B, int H, int N, float scale, int causal,
+                         cudaStream_t stream) {
+    using C = FwdCfg<D>;
+    CUtensorMap mq, mk, mv;
+    const uint64_t depth = static_cast<uint64_t>(B) * H;
+    if (!make_map_bf16_3d(&mq, Q, depth, N, D, FWD_BM) ||
+        !make_map_bf16_3d(&mk, K, depth, N, D, FWD_BN) ||
+        !make_map_bf16_3d(&mv, V, depth, N, D, FWD_BN))
+        return FA_ERR_CUDA;
+    const int di = (D == 128) ? 1 : 0;
+    if (!ds->fwd_attr[di]) {
+        if (cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return FA_ERR_CUDA;
+        ds->fwd_attr[di] = true;
+    }
+    FwdParams p;
+    p.O = static_cast<__nv_bfloat16*>(O);
+    p.LSE = LSE;
+    p.N = N;
+    p.n_kv_blocks = (N + FWD_BN - 1) / FWD_BN;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.causal = causal ? 1 : 0;
+    p.err = ds->err;
+    dim3 grid((N + 2 * FWD_BM - 1) / (2 * FWD_BM), H, B);
+    fa_fwd_kernel<D><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int H, int N, int d, float scale, int causal, cudaStream_t stream) {
+    if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+        return FA_ERR_INVALID_ARG;
+    fa_status st = check_shape(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    return d == 128 ? launch_forward<128>(ds, Q, K, V, O, LSE, B, H, N, scale, causal, stream)
+                    : launch_forward<64>(ds, Q, K, V, O, LSE, B, H, N, scale, causal, stream);
+}
+
+size_t fa_backward_workspace_bytes(int B, int H, int N, int d) {
+    if (check_shape(B, H, N, d, 1.f) != FA_OK) return 0;
+    return bwd_workspace_bytes(B, H, N, d);
+}
+
+fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                      const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                      int causal, cudaStream_t stream) {
+    if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace)
+        return FA_ERR_INVALID_ARG;
+    const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return FA_ERR_INVALID_ARG;
+    fa_status st = check_shape(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (workspace_bytes < bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    const int di = (d == 128) ? 1 : 0;
+    if (!ds->bwd_attr[di]) {
+        if (!bwd_set_attributes(d)) return FA_ERR_CUDA;
+        ds->bwd_attr[di] = true;
+    }
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, N, d, scale, causal,
+                      ds->err, stream)
+               ? FA_OK
+               : FA_ERR_CUDA;
+}
+
+fa_status fa_check_device_error(cudaStream_t stream, unsigned int* site) {
+    if (site) *site = 0;
+    fa_status st;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
+    if (v != 0) {
+        const uint32_t zero = 0;
+        if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+    }
+    if (site) *site = v;
+    return v ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+const char* fa_status_str(fa_status s) {
+    switch (s) {
+        case FA_OK: return "ok";
+        case FA_ERR_INVALID_ARG: return "invalid argument";
+        case FA_ERR_UNSUPPORTED: return "unsupported shape or device (needs sm_100, d in {64,128})";
+        case FA_ERR_CUDA: return "CUDA runtime error";
+        case FA_ERR_TIMEOUT: return "device-side bounded wait expired";
+    }
+    return "unknown status";
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

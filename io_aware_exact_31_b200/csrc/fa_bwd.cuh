@@ -1,0 +1,546 @@
+// fa_bwd.cuh -- exact attention backward for sm_100a (tcgen05 + TMA + TMEM).
+//
+// The gradient of <O, dO> for O = softmax(scale Q K^T [+causal]) V, computed
+// the way unite.ai "Flash Attention: Revolutionizing Transformer Efficiency"
+// (idea 2, recomputation) describes: the probabilities are not stored by the
+// forward but recomputed block by block from Q, K and the saved per-row
+// logsumexp.  With P_ij = exp(scale <q_i,k_j> - LSE_i):
+//     dV_j = sum_i P_ij dO_i            dP_ij = <dO_i, v_j>
+//     D_i  = <dO_i, O_i>                dS_ij = P_ij (dP_ij - D_i)
+//     dQ_i = scale sum_j dS_ij k_j      dK_j  = scale sum_i dS_ij q_i
+//
+// Three launches on the caller's stream:
+//   1. bwd_pre:  D_i (fp32), LSE_i * log2(e), zero the fp32 dQ accumulator
+//   2. bwd_main: one CTA per (key block of 128, head); loops over query blocks
+//   3. bwd_dq:   dQ = bf16(scale * dQacc)
+//
+// bwd_main, per query block i (the key block j is fixed per CTA):
+//   MMA1  S^T  = K_j Q_i^T            TMEM [0,128)      (lane = key)
+//   MMA2  dP^T = V_j dO_i^T           TMEM [128,256)
+//   MMA3  dV  += P^T dO_i             P^T bf16 in TMEM over S^T, dO MN-major
+//   MMA4  dK  += dS^T Q_i             dS^T bf16 in smem (K-major), Q MN-major
+//   MMA5  dQ_i = dS K_j               dS^T smem read MN-major, K MN-major
+// dQ_i goes to shared memory and is added to the fp32 accumulator with one
+// bulk reduce-add per block (the block's rows are contiguous in memory).
+// Warps: 0-7 compute (warp w: TMEM lane quarter w%4, column half w/4),
+// 8 MMA issuer (TMEM owner), 9 TMA producer, 10 dQ reducer.
+#pragma once
+
+#include <algorithm>
+
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace fa {
+
+constexpr int BWD_BM = 128;  // queries per block
+constexpr int BWD_BN = 128;  // keys per CTA
+constexpr int BWD_THREADS = 352;
+
+inline size_t round_up_128(int n) { return (static_cast<size_t>(n) + 127) / 128 * 128; }
+
+// Workspace: [D: BH*Npad f32][LSE2: BH*Npad f32][dQacc: BH*Npad*d f32]
+inline size_t bwd_workspace_bytes(int B, int H, int N, int d) {
+    const size_t rows = static_cast<size_t>(B) * H * round_up_128(N);
+    return rows * 4 * 2 + rows * static_cast<size_t>(d) * 4;
+}
+
+template <int D>
+struct BwdCfg {
+    static constexpr int TILE = 128 * D * 2;      // bf16 tile of 128 rows
+    static constexpr int QS = (D == 64) ? 2 : 1;  // Q/dO ring depth
+    static constexpr int CHUNKS = D / 64;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + TILE;
+    static constexpr int OFF_Q = OFF_V + TILE;               // QS tiles
+    static constexpr int OFF_DO = OFF_Q + QS * TILE;         // QS tiles
+    static constexpr int OFF_DS = OFF_DO + QS * TILE;        // 128x128 bf16 = 32 KB
+    static constexpr int OFF_DQ = OFF_DS + 32768;            // 128 x D fp32
+    static constexpr int OFF_VEC = OFF_DQ + 128 * D * 4;     // QS x (LSE2[128], D[128])
+    static constexpr int OFF_BAR = OFF_VEC + QS * 1024;
+    static constexpr int BAR_BYTES = 384;
+    static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
+    // TMEM columns
+    static constexpr uint32_t T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 256 + D;
+    static constexpr bool DQ_ALIAS = (D == 128);  // dQ shares the dP^T columns
+    static constexpr uint32_t T_DQ = DQ_ALIAS ? T_DPT : 256 + 2 * D;
+};
+
+struct BwdBars {
+    uint64_t kv_full;
+    uint64_t q_full[2], q_empty[2];
+    uint64_t s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_empty, dkdv_full;
+    uint64_t pair[4];
+    uint64_t dq_staged, dq_free;
+};
+
+struct BwdParams {
+    const float* Dvec;   // [BH, Npad]
+    const float* LSE2;   // [BH, Npad]
+    float* dQacc;        // [BH, Npad, d]
+    __nv_bfloat16* dK;
+    __nv_bfloat16* dV;
+    int N, Npad, n_q_blocks;
+    float scale, scale_log2;
+    int causal;
+    uint32_t* err;
+};
+
+// ---------------------------------------------------------------------------
+// 1. preprocess
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
+                  const float* __restrict__ LSE, float* __restrict__ Dvec,
+                  float* __restrict__ LSE2, float* __restrict__ dQacc, int N, int Npad,
+                  long long rows_pad) {
+    constexpr int TPR = D / 8;  // threads per row, 8 bf16 (16 B) each
+    const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int sub = threadIdx.x % TPR;
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x / TPR;
+    for (long long r = tid / TPR; r < rows_pad; r += stride) {
+        const long long bh = r / Npad;
+        const int i = static_cast<int>(r % Npad);
+        float acc = 0.f;
+        if (i < N) {
+            const size_t off = (static_cast<size_t>(bh) * N + i) * D + sub * 8;
+            const uint4 a = *reinterpret_cast<const uint4*>(O + off);
+            const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
+            const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
+            const __nv_bfloat162* bh2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 x = __bfloat1622float2(ah[k]);
+                const float2 y = __bfloat1622float2(bh2[k]);
+                acc = fmaf(x.x, y.x, acc);
+                acc = fmaf(x.y, y.y, acc);
+            }
+        }
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o, TPR);
+        if (sub == 0) {
+            Dvec[r] = acc;
+            LSE2[r] = (i < N) ? LSE[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : 0.f;
+        }
+        float4* z = reinterpret_cast<float4*>(dQacc + static_cast<size_t>(r) * D);
+#pragma unroll
+        for (int k = 0; k < D / 4 / TPR; ++k) z[sub + k * TPR] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. dQ finalize
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+fa_bwd_dq_kernel(const float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dQ, int N, int Npad,
+                 float scale, long long n_vec) {
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_vec;
+         e += stride) {
+        const long long row = e / (D / 8);
+        const int c8 = static_cast<int>(e % (D / 8)) * 8;
+        const long long bh = row / N;
+        const int i = static_cast<int>(row % N);
+        const float4* src =
+            reinterpret_cast<const float4*>(dQacc + (static_cast<size_t>(bh) * Npad + i) * D + c8);
+        const float4 a = src[0], b = src[1];
+        uint4 w;
+        w.x = pack_bf16x2(a.x * scale, a.y * scale);
+        w.y = pack_bf16x2(a.z * scale, a.w * scale);
+        w.z = pack_bf16x2(b.x * scale, b.y * scale);
+        w.w = pack_bf16x2(b.z * scale, b.w * scale);
+        *reinterpret_cast<uint4*>(dQ + static_cast<size_t>(row) * D + c8) = w;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2. main kernel
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                   const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapdO,
+                   const BwdParams p) {
+    using C = BwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + sizeof(BwdBars));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const Guard g{abort_flag, p.err};
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+    const int bh = blockIdx.z * gridDim.y + blockIdx.y;
+    const int kb = blockIdx.x;  // key block; causal: block 0 has the most work and starts first
+    const int k0 = kb * BWD_BN;
+    const int i_begin = p.causal ? kb : 0;  // first query block that sees this key block
+    const int n_iter = p.n_q_blocks - i_begin;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(&bars->kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->p_full, 256);
+        mbar_init(&bars->ds_full, 256);
+        mbar_init(&bars->ds_empty, 1);
+        mbar_init(&bars->dq_full, 1);
+        mbar_init(&bars->dq_empty, 256);
+        mbar_init(&bars->dkdv_full, 1);
+        for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 64);
+        mbar_init(&bars->dq_staged, 256);
+        mbar_init(&bars->dq_free, 1);
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&mapQ);
+            tma_prefetch_desc(&mapK);
+            tma_prefetch_desc(&mapV);
+            tma_prefetch_desc(&mapdO);
+            mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
+#pragma unroll
+            for (int c = 0; c < C::CHUNKS; ++c) {
+                tma_load_3d(smem + C::OFF_K + c * 16384, &mapK, &bars->kv_full, c * 64, k0, bh);
+                tma_load_3d(smem + C::OFF_V + c * 16384, &mapV, &bars->kv_full, c * 64, k0, bh);
+            }
+            int issued = 0;
+            for (int it = 0; it < n_iter; ++it) {
+                const int s = it % C::QS;
+                const uint32_t ph = (it / C::QS) & 1;
+                const int q0 = (i_begin + it) * BWD_BM;
+                if (it >= C::QS && !mbar_wait(&bars->q_empty[s], ph ^ 1, g, 21)) break;
+                mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::TILE + 1024);
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c) {
+                    tma_load_3d(smem + C::OFF_Q + s * C::TILE + c * 16384, &mapQ, &bars->q_full[s],
+                                c * 64, q0, bh);
+                    tma_load_3d(smem + C::OFF_DO + s * C::TILE + c * 16384, &mapdO,
+                                &bars->q_full[s], c * 64, q0, bh);
+                }
+                const size_t voff = static_cast<size_t>(bh) * p.Npad + q0;
+                bulk_load(smem + C::OFF_VEC + s * 1024, p.LSE2 + voff, 512, &bars->q_full[s]);
+                bulk_load(smem + C::OFF_VEC + s * 1024 + 512, p.Dvec + voff, 512, &bars->q_full[s]);
+                issued = it + 1;
+            }
+            mbar_drain(&bars->kv_full, 0);
+            for (int it = max(0, issued - C::QS); it < issued; ++it)
+                mbar_drain(&bars->q_full[it % C::QS], (it / C::QS) & 1);
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+            const uint32_t id_kn = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
+            const uint32_t id_q = idesc_bf16(128, D, true, true);      // dQ (A, B MN-major)
+            const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
+            const uint32_t sDS = smem_u32(smem + C::OFF_DS);
+            bool ok = mbar_wait(&bars->kv_full, 0, g, 22);
+            for (int it = 0; ok && it < n_iter; ++it) {
+                const int s = it % C::QS;
+                const uint32_t ph = (it / C::QS) & 1;
+                const uint32_t sQ = smem_u32(smem + C::OFF_Q + s * C::TILE);
+                const uint32_t sdO = smem_u32(smem + C::OFF_DO + s * C::TILE);
+                if (!(ok = mbar_wait(&bars->q_full[s], ph, g, 23))) break;
+                tc_fence_after();
+                // MMA1: S^T = K Q^T
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
+                    mma_ss(tmem + C::T_ST, sdesc_sw128(sK + ko, 16, 1024),
+                           sdesc_sw128(sQ + ko, 16, 1024), id_s, kk > 0);
+                }
+                tc_commit(&bars->s_full);
+                // MMA2: dP^T = V dO^T (its columns also hold dQ when aliased)
+                if (C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 24)))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
+                    mma_ss(tmem + C::T_DPT, sdesc_sw128(sV + ko, 16, 1024),
+                           sdesc_sw128(sdO + ko, 16, 1024), id_s, kk > 0);
+                }
+                tc_commit(&bars->dp_full);
+                // MMA3: dV += P^T dO   (P^T from TMEM)
+                if (!(ok = mbar_wait(&bars->p_full, it & 1, g, 25))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + C::T_DV, tmem + C::T_ST + kk * 8,
+                           sdesc_sw128(sdO + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
+                // MMA4: dK += dS^T Q
+                if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 26))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+                           sdesc_sw128(sQ + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
+                // MMA5: dQ = dS K
+                if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 27)))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + C::T_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                           sdesc_sw128(sK + kk * 2048, 16384, 1024), id_q, kk > 0);
+                tc_commit(&bars->dq_full);
+                tc_commit(&bars->ds_empty);
+                tc_commit(&bars->q_empty[s]);
+            }
+            if (ok) tc_commit(&bars->dkdv_full);
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ dQ reducer
+        if (lane == 0) {
+            const uint8_t* sDQ = smem + C::OFF_DQ;
+            for (int it = 0; it < n_iter; ++it) {
+                if (!mbar_wait(&bars->dq_staged, it & 1, g, 28)) break;
+                const int q0 = (i_begin + it) * BWD_BM;
+                bulk_reduce_add_f32(p.dQacc + (static_cast<size_t>(bh) * p.Npad + q0) * D, sDQ,
+                                    128 * D * 4);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(&bars->dq_free);
+            }
+            bulk_wait_all();
+        }
+    } else {
+        // ------------------------------------------------------------ compute warps 0-7
+        const uint32_t quarter = warp % 4, half = warp / 4;
+        const uint32_t lane_base = quarter * 32;
+        const int r = lane_base + lane;  // key row in the block (TMEM lane)
+        const int key = k0 + r;
+        const float sl2 = p.scale_log2;
+        uint8_t* sDSb = smem + C::OFF_DS + half * 16384;  // atom with queries [64*half, +64)
+        float* sDQ = reinterpret_cast<float*>(smem + C::OFF_DQ);
+        bool ok = true;
+        for (int it = 0; it < n_iter; ++it) {
+            const int s = it % C::QS;
+            const uint32_t ph = (it / C::QS) & 1;
+            const int q0 = (i_begin + it) * BWD_BM;
+            const int qh = q0 + 64 * half;  // first query of this warp's columns
+            const float* vLSE2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 1024) + 64 * half;
+            const float* vD = vLSE2 + 128;
+            // ---- P^T = exp2(S^T * scale*log2e - LSE2[q])
+            if (!(ok = mbar_wait(&bars->q_full[s], ph, g, 29))) break;
+            if (!(ok = mbar_wait_warp(&bars->s_full, it & 1, g, 30))) break;
+            tc_fence_after();
+            float pv[64];
+            {
+                uint32_t u[64];
+                tmem_ld32(tmem_addr(tmem, lane_base, C::T_ST + 64 * half), u);
+                tmem_ld32(tmem_addr(tmem, lane_base, C::T_ST + 64 * half + 32), u + 32);
+                tmem_ld_wait();
+                reg_fence<64>(u);
+#pragma unroll
+                for (int c = 0; c < 64; ++c) pv[c] = __uint_as_float(u[c]);
+            }
+            const bool need_mask = (key >= p.N) || (q0 + BWD_BM > p.N) || (p.causal && qh < k0 + BWD_BN);
+            if (need_mask) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const int q = qh + c;
+                    const bool valid = (key < p.N) && (q < p.N) && !(p.causal && key > q);
+                    pv[c] = valid ? ex2_approx(fmaf(pv[c], sl2, -vLSE2[c])) : 0.f;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) pv[c] = ex2_approx(fmaf(pv[c], sl2, -vLSE2[c]));
+            }
+            // Both column halves of these lanes must have read S^T before P^T
+            // (which overlaps it) is written.
+            mbar_arrive(&bars->pair[quarter]);
+            if (!(ok = mbar_wait_warp(&bars->pair[quarter], it & 1, g, 31))) break;
+            {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+                tmem_st32(tmem_addr(tmem, lane_base, C::T_ST + 32 * half), pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+            // ---- dS^T = P^T * (dP^T - D[q])
+            if (!(ok = mbar_wait_warp(&bars->dp_full, it & 1, g, 32))) break;
+            tc_fence_after();
+            {
+                uint32_t u[64];
+                tmem_ld32(tmem_addr(tmem, lane_base, C::T_DPT + 64 * half), u);
+                tmem_ld32(tmem_addr(tmem, lane_base, C::T_DPT + 64 * half + 32), u + 32);
+                tmem_ld_wait();
+                reg_fence<64>(u);
+#pragma unroll
+                for (int c = 0; c < 64; ++c) pv[c] = pv[c] * (__uint_as_float(u[c]) - vD[c]);
+            }
+            tc_fence_before();
+            if (it > 0 && !(ok = mbar_wait(&bars->ds_empty, (it - 1) & 1, g, 33))) break;
+            {
+                const uint32_t rowaddr = smem_u32(sDSb) + r * 128;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint32_t a = pack_bf16x2(pv[8 * cc + 0], pv[8 * cc + 1]);
+                    const uint32_t b = pack_bf16x2(pv[8 * cc + 2], pv[8 * cc + 3]);
+                    const uint32_t c2 = pack_bf16x2(pv[8 * cc + 4], pv[8 * cc + 5]);
+                    const uint32_t d2 = pack_bf16x2(pv[8 * cc + 6], pv[8 * cc + 7]);
+                    st_shared_v4(rowaddr + ((cc ^ (r & 7)) << 4), a, b, c2, d2);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->ds_full);
+            // ---- dQ_i readout (lane = query), staged for the bulk reduce
+            if (!(ok = mbar_wait_warp(&bars->dq_full, it & 1, g, 34))) break;
+            tc_fence_after();
+            constexpr int HC = D / 2;  // columns of dQ this warp reads
+            uint32_t u[HC];
+#pragma unroll
+            for (int c = 0; c < HC; c += 32)
+                tmem_ld32(tmem_addr(tmem, lane_base, C::T_DQ + HC * half + c), u + c);
+            tmem_ld_wait();
+            reg_fence<HC>(u);
+            tc_fence_before();
+            mbar_arrive(&bars->dq_empty);
+            if (it > 0 && !(ok = mbar_wait(&bars->dq_free, (it - 1) & 1, g, 35))) break;
+            {
+                float* rowp = sDQ + static_cast<size_t>(r) * D + HC * half;
+#pragma unroll
+                for (int v = 0; v < HC / 4; ++v) {
+                    const int cc = (v + lane) % (HC / 4);  // rotate to spread banks
+                    reinterpret_cast<uint4*>(rowp)[cc] =
+                        make_uint4(u[4 * cc], u[4 * cc + 1], u[4 * cc + 2], u[4 * cc + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->dq_staged);
+        }
+        // ---- dK, dV epilogue (lane = key)
+        if (ok && mbar_wait_warp(&bars->dkdv_full, 0, g, 36)) {
+            tc_fence_after();
+            constexpr int HC = D / 2;
+            const bool valid = key < p.N;
+            const size_t off = (static_cast<size_t>(bh) * p.N + (valid ? key : 0)) * D + HC * half;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = (which == 0 ? C::T_DV : C::T_DK) + HC * half;
+                const float mul = which == 0 ? 1.f : p.scale;
+                __nv_bfloat16* dst = (which == 0 ? p.dV : p.dK) + off;
+#pragma unroll
+                for (int c = 0; c < HC; c += 32) {
+                    uint32_t u[32];
+                    tmem_ld32(tmem_addr(tmem, lane_base, col + c), u);
+                    tmem_ld_wait();
+                    reg_fence<32>(u);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        w[k] = pack_bf16x2(__uint_as_float(u[2 * k]) * mul,
+                                           __uint_as_float(u[2 * k + 1]) * mul);
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            st_global_v4(dst + c + 8 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2],
+                                         w[4 * v + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+inline bool bwd_set_attributes(int d) {
+    if (d == 64)
+        return cudaFuncSetAttribute(fa_bwd_main_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
+    return cudaFuncSetAttribute(fa_bwd_main_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                BwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+}
+
+template <int D>
+bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
+                  int N, float scale, int causal, uint32_t* err, cudaStream_t stream) {
+    const int Npad = static_cast<int>(round_up_128(N));
+    const long long rows_pad = static_cast<long long>(B) * H * Npad;
+    float* Dvec = static_cast<float*>(workspace);
+    float* LSE2 = Dvec + rows_pad;
+    float* dQacc = LSE2 + rows_pad;
+    {
+        const long long threads = rows_pad * (D / 8);
+        const int blocks = static_cast<int>(std::min<long long>((threads + 255) / 256, 148LL * 16));
+        fa_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, Dvec,
+            LSE2, dQacc, N, Npad, rows_pad);
+        if (cudaGetLastError() != cudaSuccess) return false;
+    }
+    {
+        CUtensorMap mq, mk, mv, mdo;
+        const uint64_t depth = static_cast<uint64_t>(B) * H;
+        if (!make_map_bf16_3d(&mq, Q, depth, N, D, 128) || !make_map_bf16_3d(&mk, K, depth, N, D, 128) ||
+            !make_map_bf16_3d(&mv, V, depth, N, D, 128) || !make_map_bf16_3d(&mdo, dO, depth, N, D, 128))
+            return false;
+        BwdParams p;
+        p.Dvec = Dvec;
+        p.LSE2 = LSE2;
+        p.dQacc = dQacc;
+        p.dK = static_cast<__nv_bfloat16*>(dK);
+        p.dV = static_cast<__nv_bfloat16*>(dV);
+        p.N = N;
+        p.Npad = Npad;
+        p.n_q_blocks = Npad / 128;
+        p.scale = scale;
+        p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+        p.causal = causal ? 1 : 0;
+        p.err = err;
+        dim3 grid(Npad / 128, H, B);
+        fa_bwd_main_kernel<D><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+        if (cudaGetLastError() != cudaSuccess) return false;
+    }
+    {
+        const long long n_vec = static_cast<long long>(B) * H * N * (D / 8);
+        const int blocks = static_cast<int>(std::min<long long>((n_vec + 255) / 256, 148LL * 16));
+        fa_bwd_dq_kernel<D><<<blocks, 256, 0, stream>>>(dQacc, static_cast<__nv_bfloat16*>(dQ), N,
+                                                        Npad, scale, n_vec);
+        if (cudaGetLastError() != cudaSuccess) return false;
+    }
+    return true;
+}
+
+inline bool bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                       const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
+                       int N, int d, float scale, int causal, uint32_t* err, cudaStream_t stream) {
+    return d == 128 ? bwd_launch_t<128>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, N, scale,
+                                        causal, err, stream)
+                    : bwd_launch_t<64>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, N, scale,
+                                       causal, err, stream);
+}
+
+}  // namespace fa

@@ -1,0 +1,367 @@
+// fa_fwd.cuh -- exact attention forward for sm_100a (tcgen05 + TMA + TMEM).
+//
+// Computes, per head and query row i,
+//     O_i   = sum_j softmax_j(scale * <q_i, k_j>) v_j     (keys j > i masked if causal)
+//     LSE_i = ln sum_j exp(scale * <q_i, k_j>)
+// the standard-attention definition of unite.ai "Flash Attention:
+// Revolutionizing Transformer Efficiency", evaluated the IO-aware way the same
+// page describes ("Flash Attention algorithm": Q/K/V split into blocks that fit
+// in on-chip memory, two nested loops, running max m and running sum l) with
+// the merge rule of its "math behind Flash Attention" section applied block by
+// block, so the N x N score matrix never reaches HBM.  FlashAttention-2's
+// changes (systems-analysis.info "FlashAttention-2 (VI)", technical
+// architecture items 1-3) map onto this kernel as: 1) the 1/l normalisation is
+// deferred to the epilogue and one LSE per row is kept; 2) a head is split
+// over CTAs by query block; 3) warps are specialised so that a softmax row
+// lives in one thread and needs no shared-memory exchange.
+//
+// CTA = 2 query tiles of 128 rows (256 rows) of one (batch, head).
+//   warps 0-3  softmax warpgroup for tile 0 (thread = one query row = one TMEM lane)
+//   warps 4-7  softmax warpgroup for tile 1
+//   warp  8    tcgen05.mma issuer; owns the TMEM allocation
+//   warp  9    TMA producer (Q once, then the K/V ring)
+// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D)
+//   P_t (bf16, two per column) overwrites the first 64 columns of S_t and is
+//   read by the P.V MMA straight from TMEM.
+// Tensor-core issue order per key block j (P aliasing S requires PV_t(j-1)
+// before S_t(j); tcgen05 ops of one thread execute in order):
+//   PV0(j-1) S0(j) PV1(j-1) S1(j)
+// so softmax of tile 0 overlaps the tile-1 GEMMs and vice versa, and the
+// commit that publishes S_t(j) also guarantees PV_t(j-1) is complete, which is
+// when the softmax warps may rescale O_t in place.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int FWD_BM = 128;          // query rows per tile (= TMEM lanes)
+constexpr int FWD_BN = 128;          // keys per block
+constexpr int FWD_THREADS = 320;     // 10 warps
+constexpr float FWD_RESCALE_TAU = 8.0f;  // log2 units: keep a stale row max while p <= 2^8
+
+template <int D>
+struct FwdCfg {
+    static constexpr int TILE_BYTES = FWD_BM * D * 2;  // one Q, K or V tile (bf16)
+    static constexpr int NSTAGE = (D == 128) ? 2 : 3;  // K/V ring depth
+    static constexpr int CHUNKS = D / 64;              // 64-wide (128 B) TMA boxes per tile
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + NSTAGE * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NSTAGE * TILE_BYTES;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
+    static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
+};
+
+struct FwdParams {
+    __nv_bfloat16* O;
+    float* LSE;
+    int N;              // sequence length
+    int n_kv_blocks;    // ceil(N / 128)
+    float scale_log2;   // scale * log2(e)
+    int causal;
+    uint32_t* err;      // device error word
+};
+
+// Barrier slots inside the barrier area.
+struct FwdBars {
+    uint64_t q_full;
+    uint64_t k_full[3], k_empty[3];
+    uint64_t v_full[3], v_empty[3];
+    uint64_t s_full[2], p_full[2], o_full[2];
+};
+
+template <int D>
+__global__ void __launch_bounds__(FWD_THREADS, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+              const __grid_constant__ CUtensorMap mapV, const FwdParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + sizeof(FwdBars));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const Guard g{abort_flag, p.err};
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+    const int bh = blockIdx.z * gridDim.y + blockIdx.y;
+    // Causal: launch the heaviest (last) query pairs first.
+    const int pair = p.causal ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
+    const int q0 = pair * 2 * FWD_BM;
+    // Key blocks each tile needs: causal tiles stop at their diagonal block.
+    int n_tile[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int last_row = q0 + (t + 1) * FWD_BM - 1;
+        n_tile[t] = p.causal ? min(last_row / FWD_BN + 1, p.n_kv_blocks) : p.n_kv_blocks;
+    }
+    const int n_blocks = n_tile[1];  // n_tile[0] <= n_tile[1] <= n_tile[0] + 1
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars->s_full[t], 1);
+            mbar_init(&bars->p_full[t], 128);
+            mbar_init(&bars->o_full[t], 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&mapQ);
+            tma_prefetch_desc(&mapK);
+            tma_prefetch_desc(&mapV);
+            mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(smem + C::OFF_Q + t * C::TILE_BYTES + c * 16384, &mapQ,
+                                &bars->q_full, c * 64, q0 + t * FWD_BM, bh);
+            int k_issued = 0, v_issued = 0;
+            for (int j = 0; j < n_blocks; ++j) {
+                const int s = j % C::NSTAGE;
+                const uint32_t ph = (j / C::NSTAGE) & 1;
+                if (j >= C::NSTAGE && !mbar_wait(&bars->k_empty[s], ph ^ 1, g, 1)) break;
+                mbar_arrive_expect_tx(&bars->k_full[s], C::TILE_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(smem + C::OFF_K + s * C::TILE_BYTES + c * 16384, &mapK,
+                                &bars->k_full[s], c * 64, j * FWD_BN, bh);
+                k_issued = j + 1;
+                if (j >= C::NSTAGE && !mbar_wait(&bars->v_empty[s], ph ^ 1, g, 2)) break;
+                mbar_arrive_expect_tx(&bars->v_full[s], C::TILE_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::CHUNKS; ++c)
+                    tma_load_3d(smem + C::OFF_V + s * C::TILE_BYTES + c * 16384, &mapV,
+                                &bars->v_full[s], c * 64, j * FWD_BN, bh);
+                v_issued = j + 1;
+            }
+            // Never leave the CTA with copies still landing in its shared
+            // memory: wait (bounded) for the last load issued into each slot.
+            mbar_drain(&bars->q_full, 0);
+            for (int j = max(0, k_issued - C::NSTAGE); j < k_issued; ++j)
+                mbar_drain(&bars->k_full[j % C::NSTAGE], (j / C::NSTAGE) & 1);
+            for (int j = max(0, v_issued - C::NSTAGE); j < v_issued; ++j)
+                mbar_drain(&bars->v_full[j % C::NSTAGE], (j / C::NSTAGE) & 1);
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16(128, FWD_BN, false, false);  // S = Q K^T
+            const uint32_t idO = idesc_bf16(128, D, false, true);        // O += P V (V MN-major)
+            const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+            const uint32_t sK = smem_u32(smem + C::OFF_K);
+            const uint32_t sV = smem_u32(smem + C::OFF_V);
+            const uint32_t tS[2] = {tmem + C::TMEM_S0, tmem + C::TMEM_S1};
+            const uint32_t tO[2] = {tmem + C::TMEM_O0, tmem + C::TMEM_O1};
+
+            // S_t = Q_t K_j^T : K-major A and B, D/16 steps of k = 16.
+            auto issue_S = [&](int t, int s) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
+                    const uint64_t a = sdesc_sw128(sQ + t * C::TILE_BYTES + koff, 16, 1024);
+                    const uint64_t b = sdesc_sw128(sK + s * C::TILE_BYTES + koff, 16, 1024);
+                    mma_ss(tS[t], a, b, idS, kk > 0);
+                }
+            };
+            // O_t (+)= P_t V_j : P from TMEM (8 columns per k = 16), V MN-major.
+            auto issue_PV = [&](int t, int s, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < FWD_BN / 16; ++kk) {
+                    const uint64_t b = sdesc_sw128(sV + s * C::TILE_BYTES + kk * 2048, 16384, 1024);
+                    mma_ts(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+
+            bool ok = mbar_wait(&bars->q_full, 0, g, 3) && mbar_wait(&bars->k_full[0], 0, g, 4);
+            if (ok) {
+                tc_fence_after();
+                issue_S(0, 0);
+                tc_commit(&bars->s_full[0]);
+                issue_S(1, 0);
+                tc_commit(&bars->s_full[1]);
+                tc_commit(&bars->k_empty[0]);
+            }
+            for (int j = 1; ok && j <= n_blocks; ++j) {
+                // Finish block j-1 (P.V) for both tiles, then start block j (S).
+                const int sp = (j - 1) % C::NSTAGE;
+                const uint32_t php = ((j - 1) / C::NSTAGE) & 1;
+                const int s = j % C::NSTAGE;
+                const uint32_t ph = (j / C::NSTAGE) & 1;
+                const bool more = j < n_blocks;
+                if (more && !(ok = mbar_wait(&bars->k_full[s], ph, g, 5))) break;
+                if (!(ok = mbar_wait(&bars->v_full[sp], php, g, 6))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (j - 1 < n_tile[t]) {
+                        if (!(ok = mbar_wait(&bars->p_full[t], (j - 1) & 1, g, 7 + t))) break;
+                        tc_fence_after();
+                        issue_PV(t, sp, j > 1);
+                        if (j == n_tile[t]) tc_commit(&bars->o_full[t]);
+                    }
+                    if (more && j < n_tile[t]) {
+                        issue_S(t, s);
+                        tc_commit(&bars->s_full[t]);
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&bars->v_empty[sp]);
+                if (more) tc_commit(&bars->k_empty[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = warp / 4;                    // tile
+        const uint32_t lane_base = (warp % 4) * 32;  // TMEM lane quarter of this warp
+        const int row = lane_base + lane;          // row inside the tile
+        const int q = q0 + t * FWD_BM + row;       // query index
+        const uint32_t tS = tmem_addr(tmem, lane_base, t == 0 ? C::TMEM_S0 : C::TMEM_S1);
+        const uint32_t tO = tmem_addr(tmem, lane_base, t == 0 ? C::TMEM_O0 : C::TMEM_O1);
+        const float sl2 = p.scale_log2;
+        float m_used = -INFINITY;  // running row max, log2 units of scaled scores
+        float l = 0.f;             // running row sum of exp2(s*sl2 - m_used) (for LSE)
+        float lr = 0.f;            // same sum over the bf16-rounded weights (for O)
+        bool ok = true;
+        const int nt = n_tile[t];
+        const int tile_first_q = q0 + t * FWD_BM;
+        for (int j = 0; j < nt; ++j) {
+            if (!(ok = mbar_wait_warp(&bars->s_full[t], j & 1, g, 9 + t))) break;
+            tc_fence_after();
+            uint32_t sr[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+            tmem_ld_wait();
+            reg_fence<128>(sr);
+            float s[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+            const int key0 = j * FWD_BN;
+            // Mask keys past the end and (causal) keys after the query.
+            const bool tail = key0 + FWD_BN > p.N;
+            const bool diag = p.causal && key0 + FWD_BN - 1 > tile_first_q;
+            if (tail || diag) {
+                const int lim = p.causal ? min(q + 1, p.N) : p.N;  // valid keys: key < lim
+#pragma unroll
+                for (int i = 0; i < 128; ++i)
+                    if (key0 + i >= lim) s[i] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+            const float m_blk = mx * sl2;
+            float alpha = 1.f;
+            if (j == 0) {
+                m_used = m_blk;
+            } else if (m_blk > m_used + FWD_RESCALE_TAU) {
+                alpha = ex2_approx(m_used - m_blk);
+                m_used = m_blk;
+            }
+            // A row whose keys are all masked so far keeps m = -inf; use 0 so
+            // exp2(-inf - 0) = 0 instead of NaN.
+            const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+            // Rescale O_t in place when this row's max moved (rare after the
+            // first blocks).  PV_t(j-1) is complete: it was issued before S_t(j).
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_ld_wait();
+                    reg_fence<32>(o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + c * 32, o);
+                }
+            }
+            l *= alpha;
+            lr *= alpha;
+            // p = exp2(s * scale_log2 - m), rounded to bf16 for the P.V product.
+            // Two row sums: the exact one (for LSE) and one over the SAME rounded
+            // weights the tensor core multiplies V with, used to normalise O, so
+            // that O = sum p~ v / sum p~ is an exact convex combination of value
+            // rows (a row dominated by one key returns that value row exactly).
+            // P goes to TMEM as bf16 pairs (key 2c in the low half of column c).
+            float rs = 0.f, rr = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = ex2_approx(fmaf(s[h * 64 + 2 * i], sl2, -m_sub));
+                    const float p1 = ex2_approx(fmaf(s[h * 64 + 2 * i + 1], sl2, -m_sub));
+                    pk[i] = pack_bf16x2(p0, p1);
+                    rs += p0 + p1;
+                    rr += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+                }
+                tmem_st32(tS + h * 32, pk);
+            }
+            l += rs;
+            lr += rr;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[t]);
+        }
+        // ------------------------------------------------------------ epilogue
+        if (ok && mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t)) {
+            tc_fence_after();
+            const float inv_l = 1.f / lr;
+            const bool valid = q < p.N;
+            __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + (valid ? q : 0)) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_ld_wait();
+                reg_fence<32>(o);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                                       __uint_as_float(o[2 * i + 1]) * inv_l);
+                if (valid) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        st_global_v4(orow + c * 32 + v * 8, w[4 * v], w[4 * v + 1], w[4 * v + 2],
+                                     w[4 * v + 3]);
+                }
+            }
+            if (valid) {
+                // LSE in natural-log units: (m + log2 l) * ln 2.
+                p.LSE[static_cast<size_t>(bh) * p.N + q] = (m_used + __log2f(l)) * 0.69314718055994531f;
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace fa

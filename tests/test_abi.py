@@ -1,0 +1,91 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/fa.h declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from io_aware_exact_31_b200 import binding
+from io_aware_exact_31_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "fa.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert set(binding.EXPORTS) <= set(names), names
+
+
+def test_every_declared_function_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (fa_[a-z_0-9]+)\b", out))
+    for name in declared_functions():
+        assert name in exported, f"{name} declared in include/fa.h but not exported"
+        assert hasattr(lib, name)
+
+
+def test_library_does_not_link_the_oracle(lib):
+    out = subprocess.run(["nm", "-D", binding.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    assert "oracle_" not in out
+
+
+def test_status_strings(lib):
+    for st in range(5):
+        assert lib.fa_status_str(st)
+    assert lib.fa_version() >= 100
+
+
+def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64, scale=0.125, causal=0):
+    return lib.fa_forward(q, k, v, o, lse, B, H, N, d, scale, causal, None)
+
+
+def test_forward_rejects_bad_arguments_without_a_device(lib):
+    assert _fwd(lib, q=None) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, lse=None) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, v=24) == binding.FA_ERR_INVALID_ARG          # not 16-byte aligned
+    assert _fwd(lib, N=0) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, B=-1) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=-1.0) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("inf")) == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, d=96) == binding.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256) == binding.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, B=1 << 20, H=1 << 10, N=4096) == binding.FA_ERR_UNSUPPORTED
+
+
+def test_backward_rejects_bad_arguments_without_a_device(lib):
+    p = [16] * 10
+
+    def bwd(ptrs=p, ws=1 << 30, B=1, H=1, N=8, d=64, scale=0.125):
+        return lib.fa_backward(*ptrs, ws, B, H, N, d, scale, 0, None)
+
+    assert bwd(ptrs=[None] + p[1:]) == binding.FA_ERR_INVALID_ARG
+    assert bwd(ptrs=p[:9] + [None]) == binding.FA_ERR_INVALID_ARG
+    assert bwd(ptrs=p[:3] + [8] + p[4:]) == binding.FA_ERR_INVALID_ARG
+    assert bwd(ws=16) == binding.FA_ERR_INVALID_ARG
+    assert bwd(d=32) == binding.FA_ERR_UNSUPPORTED
+    assert bwd(N=0) == binding.FA_ERR_INVALID_ARG
+
+
+def test_workspace_size_formula(lib):
+    # D and LSE2 (fp32) plus the fp32 dQ accumulator, rows padded to 128 per head
+    assert lib.fa_backward_workspace_bytes(2, 3, 200, 64) == 2 * 3 * 256 * (4 + 4 + 64 * 4)
+    assert lib.fa_backward_workspace_bytes(1, 1, 128, 128) == 128 * (8 + 512)
+    assert lib.fa_backward_workspace_bytes(1, 1, 0, 64) == 0

@@ -459,3 +459,16 @@ def test_mutants_are_caught(name):
         assert caught, f"mutant {name} passed every pin"
     finally:
         shutil.rmtree(tmp, ignore_errors=True)
+
+
+def test_bf16_rounding_allowance_is_the_format_half_ulp():
+    """The O band is applied beyond |bf16(O_ref) - O_ref|; that distance is at
+    most half a bf16 ulp (1/32 for |x| in [8, 16), 1/512 for [1, 2))."""
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from _parity import bf16_rounding_distance
+    x = np.array([8.09199975993264, 1.0 + 2 ** -9, 1.0, -3.3, 12.0 + 2 ** -5])
+    dist = bf16_rounding_distance(x)
+    assert abs(dist[0] - 0.029499759932640757) < 1e-12
+    assert dist[1] == 2 ** -9 and dist[2] == 0.0 and dist[4] == 2 ** -5
+    assert np.all(dist <= np.exp2(np.floor(np.log2(np.abs(x))) - 8) + 1e-15)
