@@ -1,0 +1,409 @@
+"""Benchmark: exact attention forward (and backward) TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one forward pass (all steps of the forward path in one kernel
+launch) over the 4x16x4096x128 non-causal workload, inputs resident in HBM.
+The JSON line also reports the 16384-token causal forward and the
+forward+backward workload (backward timed alone) as extra sub-objects, a
+roofline entry for the forward kernel, SM clocks sampled during the timed
+region, an end-to-end number through the C ABI with host buffers (pinned
+host -> device copies and the device -> host read of O and LSE inside the
+timed region) and the fp64 oracle timed on a bounded sample on the host.
+
+FLOP convention: forward 4*B*H*N^2*d, halved when causal; backward 2.5x that.
+Multi-GPU (torchrun): every rank runs its own copy of the workload (heads are
+independent -- no collective on the data path); value = all ranks' FLOPs /
+the slowest rank's time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused attention fwd/bwd TFLOP/s and % of B200 dense-BF16 tensor-core peak"
+UNIT = "TFLOP/s"
+HEADLINE = "b4_h16_n4096_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha1()
+    for name in ("fa_fwd.cuh", "sm100.cuh"):
+        with open(os.path.join(ROOT, "io_aware_exact_31_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic():
+    """DRAM bytes per forward launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "fwd_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_source_sha1_12") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def time_region(fn, steps, stream, sync):
+    """CUDA-event time of `steps` calls on `stream`, bracketed by sync()."""
+    import torch
+    sync()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    sync()
+    return start.elapsed_time(end)  # ms
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from io_aware_exact_31_b200 import binding
+    from io_aware_exact_31_b200.workloads import WORKLOADS, workload_inputs
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    lib = binding.load_library()
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def fwd_setup(w):
+        x = workload_inputs(w, seed=rank)
+        q, k, v = (x[n].cuda() for n in ("Q", "K", "V"))
+        o = torch.empty_like(q)
+        lse = torch.empty(w.B, w.H, w.N, device="cuda", dtype=torch.float32)
+        args_ = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B,
+                 w.H, w.N, w.d, w.scale, int(w.causal), sh)
+        return x, (q, k, v, o, lse), args_
+
+    def launch_fwd(a):
+        st = lib.fa_forward(*a[:-1], binding.ctypes.c_void_p(a[-1]))
+        if st != 0:
+            raise binding.FaError(st, "fa_forward")
+
+    # ---------------- headline: forward on the 4x16x4096x128 workload
+    w = WORKLOADS[HEADLINE]
+    x, bufs, fargs = fwd_setup(w)
+    for _ in range(args.warmup):
+        launch_fwd(fargs)
+    with ClockSampler(local) as clk:
+        ms = time_region(lambda: launch_fwd(fargs), args.steps, stream, barrier)
+    st, site = binding.check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {site:#x}")
+    ms = max_over_ranks(ms)
+    ms_step = ms / args.steps
+    tflops = w.fwd_flops * world / (ms_step * 1e-3) / 1e12
+    per_gpu = w.fwd_flops / (ms_step * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    if args.only == "fwd":
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return {"metric": METRIC, "value": round(tflops, 1), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+                "config": {"workload": f"{HEADLINE} fwd"}, "clocks": clocks,
+                "gpu_launches": args.steps}, rank
+
+    # ---------------- e2e through the C ABI with host buffers
+    qh, kh, vh = (x[n].pin_memory() for n in ("Q", "K", "V"))
+    q, k, v, o, lse = bufs
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        launch_fwd(fargs)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    e2e_steps = max(3, args.steps // 4)
+    e2e_ms = max_over_ranks(time_region(e2e_step, e2e_steps, stream, barrier)) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    del x, bufs, fargs, qh, kh, vh, oh, lh, q, k, v, o, lse
+    torch.cuda.empty_cache()
+
+    # ---------------- extra: 16k causal forward
+    extra = {}
+    w4 = WORKLOADS["h16_n16384_d128_causal_x2"]
+    _, b4, a4 = fwd_setup(w4)
+    for _ in range(args.warmup):
+        launch_fwd(a4)
+    ms4 = max_over_ranks(time_region(lambda: launch_fwd(a4), args.steps, stream, barrier))
+    ms4 /= args.steps
+    extra[w4.name] = {"pass": "fwd", "ms": round(ms4, 4),
+                      "tflops": round(w4.fwd_flops / (ms4 * 1e-3) / 1e12, 1),
+                      "frac_of_bf16_peak": round(w4.fwd_flops / (ms4 * 1e-3) / 1e12 /
+                                                 peaks["bf16_tflops"], 4)}
+    del b4, a4
+    torch.cuda.empty_cache()
+
+    # ---------------- extra: forward + backward workload
+    w5 = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
+    x5 = workload_inputs(w5, seed=rank)
+    q5, k5, v5, do5 = (x5[n].cuda() for n in ("Q", "K", "V", "dO"))
+    o5, l5 = binding.forward(q5, k5, v5, causal=True, scale=w5.scale)
+    ws = torch.empty(binding.backward_workspace_bytes(w5.B, w5.H, w5.N, w5.d), device="cuda",
+                     dtype=torch.uint8)
+    dq5, dk5, dv5 = torch.empty_like(q5), torch.empty_like(k5), torch.empty_like(v5)
+
+    def bwd_step():
+        binding.backward(q5, k5, v5, o5, do5, l5, causal=True, scale=w5.scale, dq=dq5, dk=dk5,
+                         dv=dv5, workspace=ws)
+
+    def fwd5_step():
+        binding.forward(q5, k5, v5, causal=True, scale=w5.scale, out=o5, lse=l5)
+
+    for _ in range(args.warmup):
+        bwd_step()
+        fwd5_step()
+    msb = max_over_ranks(time_region(bwd_step, args.steps, stream, barrier)) / args.steps
+    msf = max_over_ranks(time_region(fwd5_step, args.steps, stream, barrier)) / args.steps
+    st, site = binding.check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {site:#x}")
+    extra[w5.name] = {"pass": "fwd+bwd", "fwd_ms": round(msf, 4), "bwd_ms": round(msb, 4),
+                      "fwd_tflops": round(w5.fwd_flops / (msf * 1e-3) / 1e12, 1),
+                      "bwd_tflops": round(w5.bwd_flops / (msb * 1e-3) / 1e12, 1),
+                      "bwd_launches_per_step": 3}
+
+    traffic = recorded_traffic()
+    achieved = per_gpu
+    roofline = {"bound": "tensor", "kernel": "fa_fwd_kernel<128>", "achieved": round(achieved, 1),
+                "peak": peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": traffic, "algorithmic_bytes": w.fwd_bytes,
+                "algorithmic_flops": w.fwd_flops}
+
+    result = {
+        "metric": METRIC, "value": round(tflops, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded i.i.d. N(0,1) bf16, per rank)",
+        "config": {"workload": f"{HEADLINE} fwd", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "scale": "1/sqrt(d)", "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (3 x 67 MB)"},
+        "frac_of_bf16_peak": round(per_gpu / peaks["bf16_tflops"], 4),
+        "frac_of_bf16_peak_sustained": round(per_gpu / peaks["bf16_tflops_sustained"], 4),
+        "roofline": roofline,
+        "clocks": clocks,
+        "e2e": {"value": round(w.fwd_flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "extra": extra,
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result, rank
+
+
+def oracle_sample(target_s: float, step_rows: int | None = None):
+    """Time the fp64 oracle on a bounded row sample of the headline workload.
+    Returns (tflops, seconds, rows, threads)."""
+    import numpy as np
+
+    import oracle
+    from io_aware_exact_31_b200.workloads import WORKLOADS, bf16_bits, workload_inputs
+
+    w = WORKLOADS[HEADLINE]
+    x = workload_inputs(w)
+    Q, K, V = (bf16_bits(x[n]) for n in ("Q", "K", "V"))
+    rng = np.random.default_rng(1)
+    flops_per_row = 4.0 * w.N * w.d  # non-causal
+    threads = oracle.num_threads()
+    # calibrate on a few rows, then size the sample to about target_s
+    probe = rng.choice(w.B * w.H * w.N, size=max(threads, 8), replace=False)
+    t0 = time.perf_counter()
+    oracle.attention_forward_rows(Q, K, V, w.scale, w.causal, probe)
+    dt = time.perf_counter() - t0
+    rows = step_rows or int(max(threads, min(200000, target_s / max(dt / probe.size, 1e-6))))
+    sample = rng.choice(w.B * w.H * w.N, size=rows, replace=False)
+    t0 = time.perf_counter()
+    oracle.attention_forward_rows(Q, K, V, w.scale, w.causal, sample)
+    dt = time.perf_counter() - t0
+    return flops_per_row * rows / dt / 1e12, dt, rows, threads
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return None, rank
+    # Each step times the oracle on a bounded sample (~2 s), so the whole run
+    # stays within a few minutes.
+    _, _, rows, threads = oracle_sample(2.0)
+    for _ in range(args.warmup):
+        oracle_sample(0, step_rows=max(threads, rows // 8))
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        tf, dt, r, threads = oracle_sample(0, step_rows=rows)
+        times.append(dt)
+        flops += 4.0 * 4096 * 128 * r
+    total = sum(times)
+    value = flops / total / 1e12
+    sample = (f"{rows} random query rows of {HEADLINE} per step (forward, fp64 oracle, "
+              f"full K/V of each row's head)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{HEADLINE} fwd", "B": 4, "H": 16, "N": 4096, "d": 128,
+                   "causal": False},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }, rank
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--only", default=None, choices=[None, "fwd"],
+                    help="fwd: time only the headline forward (for profiler runs)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target host time of the oracle CPU-baseline sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        res, rank = run_reference(args)
+        if rank == 0 and res is not None:
+            print(json.dumps(res))
+        return
+    # The oracle sample runs before any CUDA work (the oracle uses OpenMP
+    # threads; nothing is forked after CUDA initialisation).
+    world, rank, _ = dist_setup(args)
+    cpu = None
+    if world == 1 and rank == 0 and args.cpu_seconds > 0:
+        tf, dt, rows, threads = oracle_sample(args.cpu_seconds)
+        cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{rows} random query rows of {HEADLINE} (forward, fp64, "
+                         f"{dt:.1f} s on {threads} threads)"}
+    res, rank = run_gpu(args)
+    if rank == 0:
+        res["cpu_baseline"] = cpu
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

@@ -104,7 +104,11 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.causal = causal ? 1 : 0;
     p.err = ds->err;
-    dim3 grid((N + 2 * FWD_BM - 1) / (2 * FWD_BM), H, B);
+    p.n_heads = B * H;
+    p.n_pairs = (N + 2 * FWD_BM - 1) / (2 * FWD_BM);
+    const long long n_ctas = static_cast<long long>(p.n_pairs) * p.n_heads;
+    if (n_ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    dim3 grid(static_cast<unsigned>(n_ctas));
     fa_fwd_kernel<D><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

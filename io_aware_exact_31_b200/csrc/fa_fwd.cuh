@@ -20,6 +20,7 @@
 //   warps 4-7  softmax warpgroup for tile 1
 //   warp  8    tcgen05.mma issuer; owns the TMEM allocation
 //   warp  9    TMA producer (Q once, then the K/V ring)
+//   warps 10-11 idle (they complete the third warpgroup, which setmaxnreg needs)
 // TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D)
 //   P_t (bf16, two per column) overwrites the first 64 columns of S_t and is
 //   read by the P.V MMA straight from TMEM.
@@ -37,7 +38,12 @@ namespace fa {
 
 constexpr int FWD_BM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int FWD_BN = 128;          // keys per block
-constexpr int FWD_THREADS = 320;     // 10 warps
+constexpr int FWD_THREADS = 384;     // 12 warps = 3 warpgroups
+// Registers: launched at 168/thread (384 x 168 = 64512); the control
+// warpgroup gives back down to 56 and each softmax warpgroup takes 224:
+// 2 x 128 x 224 + 128 x 56 = 64512.
+constexpr uint32_t FWD_REGS_SOFTMAX = 224;
+constexpr uint32_t FWD_REGS_CONTROL = 56;
 constexpr float FWD_RESCALE_TAU = 8.0f;  // log2 units: keep a stale row max while p <= 2^8
 
 template <int D>
@@ -61,6 +67,8 @@ struct FwdParams {
     int n_kv_blocks;    // ceil(N / 128)
     float scale_log2;   // scale * log2(e)
     int causal;
+    int n_heads;        // B * H
+    int n_pairs;        // ceil(N / 256)
     uint32_t* err;      // device error word
 };
 
@@ -86,9 +94,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     const Guard g{abort_flag, p.err};
 
     const uint32_t warp = warp_id(), lane = lane_id();
-    const int bh = blockIdx.z * gridDim.y + blockIdx.y;
-    // Causal: launch the heaviest (last) query pairs first.
-    const int pair = p.causal ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x;
+    // 1-D grid: block b -> (pair, head) with the pair index outermost, so for
+    // causal attention the heaviest (last) query pairs of every head are
+    // dispatched first and the light ones fill the final wave.
+    const int bh = blockIdx.x % p.n_heads;
+    const int pair_rank = blockIdx.x / p.n_heads;
+    const int pair = p.causal ? (p.n_pairs - 1 - pair_rank) : pair_rank;
     const int q0 = pair * 2 * FWD_BM;
     // Key blocks each tile needs: causal tiles stop at their diagonal block.
     int n_tile[2];
@@ -124,7 +135,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 9) {
+    if (warp >= 10) {
+        // idle warps of the control warpgroup
+        regs_decrease<FWD_REGS_CONTROL>();
+    } else if (warp == 9) {
+        regs_decrease<FWD_REGS_CONTROL>();
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&mapQ);
@@ -166,6 +181,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
+        regs_decrease<FWD_REGS_CONTROL>();
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(128, FWD_BN, false, false);  // S = Q K^T
             const uint32_t idO = idesc_bf16(128, D, false, true);        // O += P V (V MN-major)
@@ -233,6 +249,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ softmax warpgroups
+        regs_increase<FWD_REGS_SOFTMAX>();
         const int t = warp / 4;                    // tile
         const uint32_t lane_base = (warp % 4) * 32;  // TMEM lane quarter of this warp
         const int row = lane_base + lane;          // row inside the tile
@@ -267,9 +284,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 for (int i = 0; i < 128; ++i)
                     if (key0 + i >= lim) s[i] = -INFINITY;
             }
-            float mx = s[0];
+            // Row max: eight independent three-input chains (short dependency depth).
+            float mx;
+            {
+                float a[8];
 #pragma unroll
-            for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+                for (int k = 0; k < 8; ++k) a[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+                for (int i = 16; i < 128; i += 16)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[i + 2 * k], s[i + 2 * k + 1]);
+                mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7]));
+            }
             const float m_blk = mx * sl2;
             float alpha = 1.f;
             if (j == 0) {
@@ -303,22 +329,31 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             // that O = sum p~ v / sum p~ is an exact convex combination of value
             // rows (a row dominated by one key returns that value row exactly).
             // P goes to TMEM as bf16 pairs (key 2c in the low half of column c).
-            float rs = 0.f, rr = 0.f;
+            // Packed f32x2 arithmetic, four independent accumulators per sum.
+            const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(-m_sub, -m_sub);
+            float2 ae[4], ar[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ae[k] = ar[k] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float p0 = ex2_approx(fmaf(s[h * 64 + 2 * i], sl2, -m_sub));
-                    const float p1 = ex2_approx(fmaf(s[h * 64 + 2 * i + 1], sl2, -m_sub));
-                    pk[i] = pack_bf16x2(p0, p1);
-                    rs += p0 + p1;
-                    rr += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+                    const float2 x =
+                        __ffma2_rn(make_float2(s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]), sl2v, negm);
+                    const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    pk[i] = pack_bf16x2(pe.x, pe.y);
+                    ae[i % 4] = __fadd2_rn(ae[i % 4], pe);
+                    ar[i % 4] = __fadd2_rn(ar[i % 4], unpack_bf16x2(pk[i]));
                 }
                 tmem_st32(tS + h * 32, pk);
             }
-            l += rs;
-            lr += rr;
+            {
+                const float2 e = __fadd2_rn(__fadd2_rn(ae[0], ae[1]), __fadd2_rn(ae[2], ae[3]));
+                const float2 r = __fadd2_rn(__fadd2_rn(ar[0], ar[1]), __fadd2_rn(ar[2], ar[3]));
+                l += e.x + e.y;
+                lr += r.x + r.y;
+            }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars->p_full[t]);
