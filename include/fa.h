@@ -92,6 +92,40 @@ fa_status fa_backward(const void *Q, const void *K, const void *V, const void *O
                       cudaStream_t stream);
 
 /*
+ * Size of the device array fa_backward_noalloc uses as its workspace (64 MiB).
+ * Every GPU on which this library's device code is loaded holds one such
+ * array until the process exits, whether or not fa_backward_noalloc is called.
+ */
+#define FA_BACKWARD_NOALLOC_MAX_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * fa_backward without a caller-supplied workspace, for callers that cannot
+ * allocate device memory: code running under a framework or engine whose
+ * allocator owns the whole device and forbids raw cudaMalloc, or a
+ * latency-critical path that cannot take the device-wide synchronisation a
+ * cudaMalloc/cudaFree may cause.  It allocates nothing: its scratch is a fixed
+ * array of FA_BACKWARD_NOALLOC_MAX_SCRATCH_BYTES inside the library (see the
+ * macro above).  The pages describe no such variant; it has no counterpart
+ * there.
+ *   Arguments, layouts and results: as fa_backward, minus the workspace.
+ *   Limit: returns FA_ERR_UNSUPPORTED, launching nothing, when
+ *     fa_backward_workspace_bytes(B,H,N,d) > FA_BACKWARD_NOALLOC_MAX_SCRATCH_BYTES
+ *     (e.g. B*H = 64 heads of N = 2048, d = 64 need 33 MiB and fit).
+ *   First call on each device: looks up the array's device address and sets
+ *     kernel attributes (host-side set-up only); make that first call before
+ *     any stream capture.
+ *   Sharing: every call on a device uses the same array.  Calls whose kernels
+ *     can overlap on the GPU (other streams, other host threads) race on it
+ *     and give undefined results; serialise them, e.g. on one stream.  Each
+ *     call first rewrites the parts of the array it reads, so leftovers from
+ *     an earlier call are harmless.
+ */
+fa_status fa_backward_noalloc(const void *Q, const void *K, const void *V, const void *O,
+                              const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
+                              int B, int H, int N, int d, float scale, int causal,
+                              cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * word.  Returns FA_OK, FA_ERR_TIMEOUT if a kernel gave up at a bounded wait
  * since the last check (its outputs are then undefined), or FA_ERR_CUDA.

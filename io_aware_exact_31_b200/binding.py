@@ -18,8 +18,11 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 
 # Every entry point include/fa.h declares.
-EXPORTS = ("fa_forward", "fa_backward_workspace_bytes", "fa_backward", "fa_check_device_error",
-           "fa_status_str", "fa_version")
+EXPORTS = ("fa_forward", "fa_backward_workspace_bytes", "fa_backward", "fa_backward_noalloc",
+           "fa_check_device_error", "fa_status_str", "fa_version")
+
+# Size of the library's built-in workspace used by fa_backward_noalloc.
+NOALLOC_MAX_SCRATCH_BYTES = 64 * 1024 * 1024
 
 _lib = None
 
@@ -47,6 +50,8 @@ def load_library(path: str | None = None):
     lib.fa_backward_workspace_bytes.restype = sz
     lib.fa_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
     lib.fa_backward.restype = i
+    lib.fa_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_backward_noalloc.restype = i
     lib.fa_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
     lib.fa_check_device_error.restype = i
     lib.fa_status_str.argtypes = [i]

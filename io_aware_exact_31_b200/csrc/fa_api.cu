@@ -193,3 +193,75 @@ const char* fa_status_str(fa_status s) {
 int fa_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fa_backward_noalloc: the backward pass with its scratch in a fixed device
+// array that lives inside this library.  For callers that must not allocate
+// device memory themselves -- code running under a framework or engine whose
+// allocator owns the whole device (a caching pool, a fixed memory budget) and
+// does not allow raw cudaMalloc, or code on a latency-critical path that
+// cannot take the device-wide synchronisation a cudaMalloc/cudaFree can
+// cause.  Nothing here allocates: the array is reserved when the library's
+// device code is loaded, on every GPU that loads it, and is released only when
+// the process exits.
+// ---------------------------------------------------------------------------
+namespace fa {
+namespace {
+
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[FA_BACKWARD_NOALLOC_MAX_SCRATCH_BYTES];
+
+struct NoallocDevice {
+    bool ready = false;
+    void* scratch = nullptr;  // device address of g_noalloc_scratch on this GPU
+};
+NoallocDevice g_noalloc[kMaxDevices];
+
+}  // namespace
+}  // namespace fa
+
+extern "C" fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V,
+                                         const void* O, const void* dO, const float* LSE,
+                                         void* dQ, void* dK, void* dV, int B, int H, int N,
+                                         int d, float scale, int causal, cudaStream_t stream) {
+    if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
+    const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return FA_ERR_INVALID_ARG;
+    fa_status st = check_shape(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    // The whole workspace must fit in the fixed array.
+    if (bwd_workspace_bytes(B, H, N, d) > FA_BACKWARD_NOALLOC_MAX_SCRATCH_BYTES)
+        return FA_ERR_UNSUPPORTED;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        NoallocDevice& nd = g_noalloc[dev];
+        if (!nd.ready) {
+            // Once per device, with that device current: in host code the
+            // array's name only stands in for it, so fetch its real address.
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+                return FA_ERR_CUDA;
+            nd.scratch = p;
+            nd.ready = true;
+        }
+        scratch = nd.scratch;
+        const int di = (d == 128) ? 1 : 0;
+        if (!ds->bwd_attr[di]) {
+            if (!bwd_set_attributes(d)) return FA_ERR_CUDA;
+            ds->bwd_attr[di] = true;
+        }
+    }
+    // Same three kernels as fa_backward; the preprocess kernel rewrites every
+    // byte of the scratch the later kernels read (D, LSE and the zeroed fp32
+    // dQ accumulator), so what an earlier call left there does not matter.
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, scratch, B, H, N, d, scale, causal,
+                      ds->err, stream)
+               ? FA_OK
+               : FA_ERR_CUDA;
+}
