@@ -58,69 +58,92 @@ def kernel_source_hash() -> str:
 def recorded_traffic():
     """DRAM bytes per forward launch from the committed ncu summary, if it was
     taken on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", "fwd_traffic.json")
+    path = os.path.join(ROOT, "profiles", "fwd_traffic.txt")
+    d = {}
     try:
         with open(path) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
+            for line in f:
+                if "=" in line and not line.lstrip().startswith("#"):
+                    k, v = line.strip().split("=", 1)
+                    d[k] = v
+    except OSError:
         return None
     if d.get("kernel_source_sha1_12") != kernel_source_hash():
         return None
-    return d.get("dram_bytes_per_launch")
+    try:
+        return int(d["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML every
+    `period` seconds by a background thread while the timed region runs."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int):
-        self.dev = device_index
-        self.proc = None
-        self.out = None
+    def __init__(self, device_index: int, period: float = 0.002):
+        self.dev, self.period = device_index, period
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = None
+        self._thr = None
+        self.error = None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self._nvml_index(pynvml))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        except Exception as e:  # noqa: BLE001 - report, don't fail the bench
+            self.error = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    for name, bit in self.REASONS.items():
+                        if r & bit:
+                            self.reasons.add(name)
+                except Exception as e:  # noqa: BLE001
+                    self.error = str(e)
+                    return
+                self._stop.wait(self.period)
+
+        self._thr = threading.Thread(target=loop, daemon=True)
+        self._thr.start()
         return self
 
+    def _nvml_index(self, pynvml):
+        # NVML numbers devices by PCI order; map the CUDA device through its bus id.
+        try:
+            import torch
+            bus = torch.cuda.get_device_properties(self.dev).pci_bus_id
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                if pynvml.nvmlDeviceGetPciInfo(hh).busId.decode().lower().endswith(bus.lower()[-12:]):
+                    return i
+        except Exception:  # noqa: BLE001
+            pass
+        return self.dev
+
     def __exit__(self, *exc):
-        if self.proc is not None:
-            time.sleep(0.2)
-            self.proc.terminate()
-            try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                self.out, _ = self.proc.communicate()
+        if self._stop is not None:
+            self._stop.set()
+            self._thr.join(timeout=2)
 
     def summary(self):
-        if not self.out:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"],
+                    "samples": 0, "note": self.error}
+        return {"sm_mhz": statistics.median(self.samples), "sm_min_mhz": min(self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "NVML, 2 ms period"}
 
 
 def dist_setup(args):
@@ -128,6 +151,22 @@ def dist_setup(args):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Maximum of x over all ranks (identity for one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tflops(flops_per_rank: float, world: int, ms_per_step_slowest: float) -> float:
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's time."""
+    return flops_per_rank * world / (ms_per_step_slowest * 1e-3) / 1e12
 
 
 def time_region(fn, steps, stream, sync):
@@ -164,12 +203,8 @@ def run_gpu(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x: float) -> float:
+        return max_over_ranks(x, world, "cuda")
 
     peaks, peak_src = load_peaks()
     lib = binding.load_library()
@@ -190,6 +225,9 @@ def run_gpu(args):
         if st != 0:
             raise binding.FaError(st, "fa_forward")
 
+    if args.only == "bwd":
+        return run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank), rank
+
     # ---------------- headline: forward on the 4x16x4096x128 workload
     w = WORKLOADS[HEADLINE]
     x, bufs, fargs = fwd_setup(w)
@@ -200,11 +238,25 @@ def run_gpu(args):
     st, site = binding.check_device_error()
     if st != 0:
         raise RuntimeError(f"device error {site:#x}")
-    ms = max_over_ranks(ms)
+    ms = max_ranks(ms)
     ms_step = ms / args.steps
-    tflops = w.fwd_flops * world / (ms_step * 1e-3) / 1e12
+    tflops = weak_scaling_tflops(w.fwd_flops, world, ms_step)
     per_gpu = w.fwd_flops / (ms_step * 1e-3) / 1e12
     clocks = clk.summary()
+
+    # ---------------- the same forward held for ~1.5 s: power-capped regime,
+    # reported against the sustained peak
+    sustained = None
+    if args.sustained_seconds > 0:
+        n_sus = max(args.steps, int(args.sustained_seconds * 1e3 / ms_step))
+        with ClockSampler(local) as clk_s:
+            ms_s = max_ranks(time_region(lambda: launch_fwd(fargs), n_sus, stream, barrier))
+        ms_s /= n_sus
+        tf_s = w.fwd_flops / (ms_s * 1e-3) / 1e12
+        sustained = {"steps": n_sus, "ms_per_step": round(ms_s, 4),
+                     "tflops_per_gpu": round(tf_s, 1),
+                     "frac_of_bf16_peak_sustained": round(tf_s / peaks["bf16_tflops_sustained"], 4),
+                     "clocks": clk_s.summary()}
 
     if args.only == "fwd":
         if world > 1:
@@ -232,7 +284,7 @@ def run_gpu(args):
     for _ in range(2):
         e2e_step()
     e2e_steps = max(3, args.steps // 4)
-    e2e_ms = max_over_ranks(time_region(e2e_step, e2e_steps, stream, barrier)) / e2e_steps
+    e2e_ms = max_ranks(time_region(e2e_step, e2e_steps, stream, barrier)) / e2e_steps
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
     del x, bufs, fargs, qh, kh, vh, oh, lh, q, k, v, o, lse
@@ -244,7 +296,7 @@ def run_gpu(args):
     _, b4, a4 = fwd_setup(w4)
     for _ in range(args.warmup):
         launch_fwd(a4)
-    ms4 = max_over_ranks(time_region(lambda: launch_fwd(a4), args.steps, stream, barrier))
+    ms4 = max_ranks(time_region(lambda: launch_fwd(a4), args.steps, stream, barrier))
     ms4 /= args.steps
     extra[w4.name] = {"pass": "fwd", "ms": round(ms4, 4),
                       "tflops": round(w4.fwd_flops / (ms4 * 1e-3) / 1e12, 1),
@@ -272,8 +324,8 @@ def run_gpu(args):
     for _ in range(args.warmup):
         bwd_step()
         fwd5_step()
-    msb = max_over_ranks(time_region(bwd_step, args.steps, stream, barrier)) / args.steps
-    msf = max_over_ranks(time_region(fwd5_step, args.steps, stream, barrier)) / args.steps
+    msb = max_ranks(time_region(bwd_step, args.steps, stream, barrier)) / args.steps
+    msf = max_ranks(time_region(fwd5_step, args.steps, stream, barrier)) / args.steps
     st, site = binding.check_device_error()
     if st != 0:
         raise RuntimeError(f"device error {site:#x}")
@@ -302,6 +354,7 @@ def run_gpu(args):
         "frac_of_bf16_peak_sustained": round(per_gpu / peaks["bf16_tflops_sustained"], 4),
         "roofline": roofline,
         "clocks": clocks,
+        "sustained": sustained,
         "e2e": {"value": round(w.fwd_flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -312,6 +365,29 @@ def run_gpu(args):
         dist.barrier()
         dist.destroy_process_group()
     return result, rank
+
+
+def run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank):
+    """Backward of the 4x16x2048x64 causal workload alone (for profiler runs)."""
+    w5 = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
+    x5 = workload_inputs(w5, seed=rank)
+    q, k, v, do = (x5[n].cuda() for n in ("Q", "K", "V", "dO"))
+    o, lse = binding.forward(q, k, v, causal=True, scale=w5.scale)
+    ws = torch.empty(binding.backward_workspace_bytes(w5.B, w5.H, w5.N, w5.d), device="cuda",
+                     dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def step():
+        binding.backward(q, k, v, o, do, lse, causal=True, scale=w5.scale, dq=dq, dk=dk, dv=dv,
+                         workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    stream = torch.cuda.current_stream()
+    ms = time_region(step, args.steps, stream, torch.cuda.synchronize) / args.steps
+    return {"metric": METRIC, "value": round(w5.bwd_flops / (ms * 1e-3) / 1e12, 1),
+            "unit": UNIT, "ms_per_step": round(ms, 4), "steps": args.steps,
+            "config": {"workload": f"{w5.name} bwd"}, "gpu_launches": 3 * args.steps}
 
 
 def oracle_sample(target_s: float, step_rows: int | None = None):
@@ -347,7 +423,7 @@ def run_reference(args):
         return None, rank
     # Each step times the oracle on a bounded sample (~2 s), so the whole run
     # stays within a few minutes.
-    _, _, rows, threads = oracle_sample(2.0)
+    _, _, rows, threads = oracle_sample(args.ref_step_seconds)
     for _ in range(args.warmup):
         oracle_sample(0, step_rows=max(threads, rows // 8))
     times, flops = [], 0.0
@@ -375,11 +451,15 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--sustained-seconds", type=float, default=1.5,
+                    help="length of the extra power-capped forward loop (0 to skip)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--only", default=None, choices=[None, "fwd"],
-                    help="fwd: time only the headline forward (for profiler runs)")
+    ap.add_argument("--ref-step-seconds", type=float, default=2.0,
+                    help="host time of one oracle step in --impl reference")
+    ap.add_argument("--only", default=None, choices=[None, "fwd", "bwd"],
+                    help="time only the headline forward / the backward (profiler runs)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target host time of the oracle CPU-baseline sample")
     args = ap.parse_args()

@@ -94,12 +94,19 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     const Guard g{abort_flag, p.err};
 
     const uint32_t warp = warp_id(), lane = lane_id();
-    // 1-D grid: block b -> (pair, head) with the pair index outermost, so for
-    // causal attention the heaviest (last) query pairs of every head are
-    // dispatched first and the light ones fill the final wave.
-    const int bh = blockIdx.x % p.n_heads;
-    const int pair_rank = blockIdx.x / p.n_heads;
-    const int pair = p.causal ? (p.n_pairs - 1 - pair_rank) : pair_rank;
+    // 1-D grid.  Causal: block b -> (pair, head) with the pair index
+    // outermost and descending, so every head's heaviest (last) query pairs
+    // are dispatched first and the light ones fill the final wave.
+    // Non-causal (all CTAs equal): head-major, the pairs of one head adjacent,
+    // so the CTAs resident at one time share few heads' K/V in L2.
+    int bh, pair;
+    if (p.causal) {
+        bh = blockIdx.x % p.n_heads;
+        pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x / p.n_heads);
+    } else {
+        bh = blockIdx.x / p.n_pairs;
+        pair = blockIdx.x % p.n_pairs;
+    }
     const int q0 = pair * 2 * FWD_BM;
     // Key blocks each tile needs: causal tiles stop at their diagonal block.
     int n_tile[2];
