@@ -133,6 +133,19 @@ fa_status fa_backward_noalloc(const void *Q, const void *K, const void *V, const
  */
 fa_status fa_check_device_error(cudaStream_t stream, unsigned int *site);
 
+/*
+ * Self-test of the failure-detection path (diagnostic; not part of the
+ * attention computation).  Enqueues on `stream` a one-CTA kernel whose first
+ * warp waits, for at most timeout_ns (1 ns .. 1 s), on a barrier that nothing
+ * ever arrives at, exactly as the attention kernels' bounded waits do; it
+ * gives up, records a timeout code in the device error word and releases the
+ * other waiting warp through the CTA abort flag.  A following
+ * fa_check_device_error must return FA_ERR_TIMEOUT with site 0x163; the CUDA
+ * context stays usable.  Returns FA_ERR_INVALID_ARG for an out-of-range
+ * timeout.
+ */
+fa_status fa_selftest_bounded_wait(unsigned long long timeout_ns, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char *fa_status_str(fa_status status);
 

@@ -19,7 +19,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 
 # Every entry point include/fa.h declares.
 EXPORTS = ("fa_forward", "fa_backward_workspace_bytes", "fa_backward", "fa_backward_noalloc",
-           "fa_check_device_error", "fa_status_str", "fa_version")
+           "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_str", "fa_version")
 
 # Size of the library's built-in workspace used by fa_backward_noalloc.
 NOALLOC_MAX_SCRATCH_BYTES = 64 * 1024 * 1024
@@ -54,6 +54,8 @@ def load_library(path: str | None = None):
     lib.fa_backward_noalloc.restype = i
     lib.fa_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
     lib.fa_check_device_error.restype = i
+    lib.fa_selftest_bounded_wait.argtypes = [ctypes.c_ulonglong, vp]
+    lib.fa_selftest_bounded_wait.restype = i
     lib.fa_status_str.argtypes = [i]
     lib.fa_status_str.restype = ctypes.c_char_p
     lib.fa_version.restype = i
@@ -139,6 +141,14 @@ def check_device_error(stream=None) -> tuple[int, int]:
     site = ctypes.c_uint(0)
     st = load_library().fa_check_device_error(_stream_handle(stream), ctypes.byref(site))
     return st, site.value
+
+
+def selftest_bounded_wait(timeout_ns: int = 20_000_000, stream=None) -> tuple[int, int]:
+    """Run the bounded-wait self-test and return check_device_error()'s result."""
+    st = load_library().fa_selftest_bounded_wait(int(timeout_ns), _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_selftest_bounded_wait")
+    return check_device_error(stream)
 
 
 class _Attention(torch.autograd.Function):

@@ -113,6 +113,31 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Self-test of the bounded-wait path: warp 0 waits, with a short limit, on a
+// barrier that nothing ever arrives at, so it gives up and records
+// DEV_TIMEOUT_BASE + SELFTEST_SITE; warp 1 waits on the same barrier with the
+// kernels' normal limit and must be released early by the abort flag.
+constexpr uint32_t SELFTEST_SITE = 0x63;
+
+__global__ void __launch_bounds__(64)
+fa_selftest_wait_kernel(uint32_t* err, unsigned long long timeout_ns, int* released) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const Guard g{&abort_flag, err};
+    bool ok;
+    if (warp_id() == 0)
+        ok = mbar_wait(&bar, 0, g, SELFTEST_SITE, timeout_ns);
+    else
+        ok = mbar_wait(&bar, 0, g, SELFTEST_SITE + 1);
+    if (!ok && warp_id() == 1 && lane_id() == 0 && released) *released = 1;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -177,6 +202,15 @@ fa_status fa_check_device_error(cudaStream_t stream, unsigned int* site) {
     }
     if (site) *site = v;
     return v ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+fa_status fa_selftest_bounded_wait(unsigned long long timeout_ns, cudaStream_t stream) {
+    if (timeout_ns == 0 || timeout_ns > 1000000000ull) return FA_ERR_INVALID_ARG;
+    fa_status st;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    fa_selftest_wait_kernel<<<1, 64, 0, stream>>>(ds->err, timeout_ns, nullptr);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 const char* fa_status_str(fa_status s) {

@@ -20,10 +20,10 @@
 //   MMA3  dV  += P^T dO_i             P^T bf16 in TMEM over S^T, dO MN-major
 //   MMA4  dK  += dS^T Q_i             dS^T bf16 in smem (K-major), Q MN-major
 //   MMA5  dQ_i = dS K_j               dS^T smem read MN-major, K MN-major
-// dQ_i goes to shared memory and is added to the fp32 accumulator with one
-// bulk reduce-add per block (the block's rows are contiguous in memory).
+// dQ_i goes to 128-B-swizzled shared memory and is added to the fp32
+// accumulator with TMA tensor reduce-adds (one per 32-column box).
 // Warps: 0-7 compute (warp w: TMEM lane quarter w%4, column half w/4),
-// 8 MMA issuer (TMEM owner), 9 TMA producer, 10 dQ reducer.
+// 8 MMA issuer (TMEM owner), 9 TMA producer, 10 dQ reducer, 11 idle.
 #pragma once
 
 #include <algorithm>
@@ -35,7 +35,11 @@ namespace fa {
 
 constexpr int BWD_BM = 128;  // queries per block
 constexpr int BWD_BN = 128;  // keys per CTA
-constexpr int BWD_THREADS = 352;
+constexpr int BWD_THREADS = 384;  // 3 warpgroups
+// Registers: launched at 168 (384 x 168 = 64512); the control warpgroup drops
+// to 72 and the two compute warpgroups rise to 216: 256 x 216 + 128 x 72.
+constexpr uint32_t BWD_REGS_COMPUTE = 216;
+constexpr uint32_t BWD_REGS_CONTROL = 72;
 
 inline size_t round_up_128(int n) { return (static_cast<size_t>(n) + 127) / 128 * 128; }
 
@@ -55,7 +59,7 @@ struct BwdCfg {
     static constexpr int OFF_Q = OFF_V + TILE;               // QS tiles
     static constexpr int OFF_DO = OFF_Q + QS * TILE;         // QS tiles
     static constexpr int OFF_DS = OFF_DO + QS * TILE;        // 128x128 bf16 = 32 KB
-    static constexpr int OFF_DQ = OFF_DS + 32768;            // 128 x D fp32
+    static constexpr int OFF_DQ = OFF_DS + 32768;            // 128 x D fp32, D/32 swizzled boxes
     static constexpr int OFF_VEC = OFF_DQ + 128 * D * 4;     // QS x (LSE2[128], D[128])
     static constexpr int OFF_BAR = OFF_VEC + QS * 1024;
     static constexpr int BAR_BYTES = 384;
@@ -63,6 +67,7 @@ struct BwdCfg {
     // TMEM columns
     static constexpr uint32_t T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 256 + D;
     static constexpr bool DQ_ALIAS = (D == 128);  // dQ shares the dP^T columns
+    static constexpr bool EARLY_S = (QS >= 2);    // issue S^T(i+1) before dK/dQ(i)
     static constexpr uint32_t T_DQ = DQ_ALIAS ? T_DPT : 256 + 2 * D;
 };
 
@@ -158,11 +163,20 @@ fa_bwd_dq_kernel(const float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dQ
 // ---------------------------------------------------------------------------
 // 2. main kernel
 // ---------------------------------------------------------------------------
+// Per query block i the compute warps do three phases:
+//   P(i):   P^T = exp2(S^T * scale*log2e - LSE2[q])  (TMEM -> regs -> TMEM)
+//   dS(i):  dS^T = P^T * (dP^T - D[q])               (-> swizzled smem, bf16)
+//   dQr(i): dQ_i from TMEM -> swizzled fp32 smem staging for the reducer warp
+// With two Q/dO stages (d = 64) the work is software-pipelined:
+//   compute:  P(0) dS(0) | P(1) dQr(0) dS(1) | P(2) dQr(1) dS(2) | ... dQr(n-1)
+//   MMA:      S(0) dP(0) dV(0) | S(1) dK(0) dQ(0) dP(1) dV(1) | S(2) dK(1) ...
+// so the exp work of block i+1 overlaps the dK/dQ MMAs of block i.  With one
+// stage (d = 128: shared memory is full) the MMAs run in plain order.
 template <int D>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapdO,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap mapdQacc, const BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -208,8 +222,11 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 9) {
+    if (warp >= 11) {
+        regs_decrease<BWD_REGS_CONTROL>();  // idle warp of the control warpgroup
+    } else if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
+        regs_decrease<BWD_REGS_CONTROL>();
         if (lane == 0) {
             tma_prefetch_desc(&mapQ);
             tma_prefetch_desc(&mapK);
@@ -246,76 +263,100 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
+        regs_decrease<BWD_REGS_CONTROL>();
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);  // S^T, dP^T
             const uint32_t id_kn = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
             const uint32_t id_q = idesc_bf16(128, D, true, true);      // dQ (A, B MN-major)
             const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
             const uint32_t sDS = smem_u32(smem + C::OFF_DS);
-            bool ok = mbar_wait(&bars->kv_full, 0, g, 22);
-            for (int it = 0; ok && it < n_iter; ++it) {
-                const int s = it % C::QS;
-                const uint32_t ph = (it / C::QS) & 1;
-                const uint32_t sQ = smem_u32(smem + C::OFF_Q + s * C::TILE);
-                const uint32_t sdO = smem_u32(smem + C::OFF_DO + s * C::TILE);
-                if (!(ok = mbar_wait(&bars->q_full[s], ph, g, 23))) break;
-                tc_fence_after();
-                // MMA1: S^T = K Q^T
+            auto sQ = [&](int it) { return smem_u32(smem + C::OFF_Q + (it % C::QS) * C::TILE); };
+            auto sdO = [&](int it) { return smem_u32(smem + C::OFF_DO + (it % C::QS) * C::TILE); };
+            auto mma_S = [&](int it) {  // S^T = K Q^T
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
                     mma_ss(tmem + C::T_ST, sdesc_sw128(sK + ko, 16, 1024),
-                           sdesc_sw128(sQ + ko, 16, 1024), id_s, kk > 0);
+                           sdesc_sw128(sQ(it) + ko, 16, 1024), id_s, kk > 0);
                 }
                 tc_commit(&bars->s_full);
-                // MMA2: dP^T = V dO^T (its columns also hold dQ when aliased)
-                if (C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 24)))
-                    break;
-                tc_fence_after();
+            };
+            auto mma_dP = [&](int it) {  // dP^T = V dO^T
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
                     mma_ss(tmem + C::T_DPT, sdesc_sw128(sV + ko, 16, 1024),
-                           sdesc_sw128(sdO + ko, 16, 1024), id_s, kk > 0);
+                           sdesc_sw128(sdO(it) + ko, 16, 1024), id_s, kk > 0);
                 }
                 tc_commit(&bars->dp_full);
-                // MMA3: dV += P^T dO   (P^T from TMEM)
-                if (!(ok = mbar_wait(&bars->p_full, it & 1, g, 25))) break;
-                tc_fence_after();
+            };
+            auto mma_dV = [&](int it) {  // dV += P^T dO   (P^T from TMEM)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tmem + C::T_DV, tmem + C::T_ST + kk * 8,
-                           sdesc_sw128(sdO + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
-                // MMA4: dK += dS^T Q
-                if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 26))) break;
-                tc_fence_after();
+                           sdesc_sw128(sdO(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
+            };
+            auto mma_dK_dQ = [&](int it) {  // dK += dS^T Q ; dQ = dS K
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
-                           sdesc_sw128(sQ + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
-                // MMA5: dQ = dS K
-                if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 27)))
-                    break;
-                tc_fence_after();
+                           sdesc_sw128(sQ(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tmem + C::T_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
                            sdesc_sw128(sK + kk * 2048, 16384, 1024), id_q, kk > 0);
                 tc_commit(&bars->dq_full);
                 tc_commit(&bars->ds_empty);
-                tc_commit(&bars->q_empty[s]);
+                tc_commit(&bars->q_empty[it % C::QS]);
+            };
+            bool ok = mbar_wait(&bars->kv_full, 0, g, 22) &&
+                      mbar_wait(&bars->q_full[0], 0, g, 23);
+            if (ok) {
+                tc_fence_after();
+                mma_S(0);
+                mma_dP(0);
+            }
+            for (int it = 0; ok && it < n_iter; ++it) {
+                const bool more = it + 1 < n_iter;
+                const int s1 = (it + 1) % C::QS;
+                const uint32_t ph1 = ((it + 1) / C::QS) & 1;
+                if (!(ok = mbar_wait(&bars->p_full, it & 1, g, 25))) break;
+                tc_fence_after();
+                mma_dV(it);
+                if (C::EARLY_S && more) {
+                    if (!(ok = mbar_wait(&bars->q_full[s1], ph1, g, 23))) break;
+                    tc_fence_after();
+                    mma_S(it + 1);
+                }
+                if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 26))) break;
+                if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 27)))
+                    break;
+                tc_fence_after();
+                mma_dK_dQ(it);
+                if (more) {
+                    if (!C::EARLY_S) {
+                        if (!(ok = mbar_wait(&bars->q_full[s1], ph1, g, 23))) break;
+                        tc_fence_after();
+                        mma_S(it + 1);
+                    }
+                    if (C::DQ_ALIAS && !(ok = mbar_wait(&bars->dq_empty, it & 1, g, 24))) break;
+                    tc_fence_after();
+                    mma_dP(it + 1);
+                }
             }
             if (ok) tc_commit(&bars->dkdv_full);
         }
     } else if (warp == 10) {
         // ------------------------------------------------------------ dQ reducer
+        regs_decrease<BWD_REGS_CONTROL>();
         if (lane == 0) {
-            const uint8_t* sDQ = smem + C::OFF_DQ;
+            tma_prefetch_desc(&mapdQacc);
             for (int it = 0; it < n_iter; ++it) {
                 if (!mbar_wait(&bars->dq_staged, it & 1, g, 28)) break;
                 const int q0 = (i_begin + it) * BWD_BM;
-                bulk_reduce_add_f32(p.dQacc + (static_cast<size_t>(bh) * p.Npad + q0) * D, sDQ,
-                                    128 * D * 4);
+#pragma unroll
+                for (int b = 0; b < D / 32; ++b)
+                    tma_reduce_add_3d(&mapdQacc, smem + C::OFF_DQ + b * 16384, b * 32, q0, bh);
                 bulk_commit_group();
                 bulk_wait_read_all();
                 mbar_arrive(&bars->dq_free);
@@ -324,26 +365,26 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         }
     } else {
         // ------------------------------------------------------------ compute warps 0-7
+        regs_increase<BWD_REGS_COMPUTE>();
         const uint32_t quarter = warp % 4, half = warp / 4;
         const uint32_t lane_base = quarter * 32;
-        const int r = lane_base + lane;  // key row in the block (TMEM lane)
+        const int r = lane_base + lane;  // TMEM lane: key row (P, dS) or query row (dQ)
         const int key = k0 + r;
         const float sl2 = p.scale_log2;
-        uint8_t* sDSb = smem + C::OFF_DS + half * 16384;  // atom with queries [64*half, +64)
-        float* sDQ = reinterpret_cast<float*>(smem + C::OFF_DQ);
+        const uint32_t sDSrow = smem_u32(smem + C::OFF_DS + half * 16384) + r * 128;
+        const uint32_t sDQ = smem_u32(smem + C::OFF_DQ);
+        float pv[64];  // P^T (then dS^T) for this thread's 64 queries
         bool ok = true;
-        for (int it = 0; it < n_iter; ++it) {
+
+        // ---- P(it): P^T = exp2(S^T * scale*log2e - LSE2[q])
+        auto phase_P = [&](int it) -> bool {
             const int s = it % C::QS;
             const uint32_t ph = (it / C::QS) & 1;
             const int q0 = (i_begin + it) * BWD_BM;
             const int qh = q0 + 64 * half;  // first query of this warp's columns
-            const float* vLSE2 = reinterpret_cast<const float*>(smem + C::OFF_VEC + s * 1024) + 64 * half;
-            const float* vD = vLSE2 + 128;
-            // ---- P^T = exp2(S^T * scale*log2e - LSE2[q])
-            if (!(ok = mbar_wait(&bars->q_full[s], ph, g, 29))) break;
-            if (!(ok = mbar_wait_warp(&bars->s_full, it & 1, g, 30))) break;
+            if (!mbar_wait(&bars->q_full[s], ph, g, 29)) return false;
+            if (!mbar_wait_warp(&bars->s_full, it & 1, g, 30)) return false;
             tc_fence_after();
-            float pv[64];
             {
                 uint32_t u[64];
                 tmem_ld32(tmem_addr(tmem, lane_base, C::T_ST + 64 * half), u);
@@ -353,22 +394,31 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
 #pragma unroll
                 for (int c = 0; c < 64; ++c) pv[c] = __uint_as_float(u[c]);
             }
-            const bool need_mask = (key >= p.N) || (q0 + BWD_BM > p.N) || (p.causal && qh < k0 + BWD_BN);
+            const uint32_t vL = smem_u32(smem + C::OFF_VEC + s * 1024) + 256 * half;
+            const bool need_mask =
+                (key >= p.N) || (q0 + BWD_BM > p.N) || (p.causal && qh < k0 + BWD_BN);
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 l4 = ld_shared_v4f(vL + 16 * c4);
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = 4 * c4 + e;
+                    pv[c] = ex2_approx(fmaf(pv[c], sl2, -lv[e]));
+                }
+            }
             if (need_mask) {
+                const int qlim = p.causal ? key : 0;   // causal: keep q >= key
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const int q = qh + c;
-                    const bool valid = (key < p.N) && (q < p.N) && !(p.causal && key > q);
-                    pv[c] = valid ? ex2_approx(fmaf(pv[c], sl2, -vLSE2[c])) : 0.f;
+                    if (key >= p.N || q >= p.N || q < qlim) pv[c] = 0.f;
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) pv[c] = ex2_approx(fmaf(pv[c], sl2, -vLSE2[c]));
             }
             // Both column halves of these lanes must have read S^T before P^T
             // (which overlaps it) is written.
             mbar_arrive(&bars->pair[quarter]);
-            if (!(ok = mbar_wait_warp(&bars->pair[quarter], it & 1, g, 31))) break;
+            if (!mbar_wait_warp(&bars->pair[quarter], it & 1, g, 31)) return false;
             {
                 uint32_t pk[32];
 #pragma unroll
@@ -378,9 +428,14 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars->p_full);
-            // ---- dS^T = P^T * (dP^T - D[q])
-            if (!(ok = mbar_wait_warp(&bars->dp_full, it & 1, g, 32))) break;
+            return true;
+        };
+        // ---- dS(it): dS^T = P^T * (dP^T - D[q]) -> swizzled bf16 smem
+        auto phase_dS = [&](int it) -> bool {
+            const int s = it % C::QS;
+            if (!mbar_wait_warp(&bars->dp_full, it & 1, g, 32)) return false;
             tc_fence_after();
+            const uint32_t vD = smem_u32(smem + C::OFF_VEC + s * 1024) + 512 + 256 * half;
             {
                 uint32_t u[64];
                 tmem_ld32(tmem_addr(tmem, lane_base, C::T_DPT + 64 * half), u);
@@ -388,27 +443,36 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
                 tmem_ld_wait();
                 reg_fence<64>(u);
 #pragma unroll
-                for (int c = 0; c < 64; ++c) pv[c] = pv[c] * (__uint_as_float(u[c]) - vD[c]);
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const float4 d4 = ld_shared_v4f(vD + 16 * c4);
+                    const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 4 * c4 + e;
+                        pv[c] = pv[c] * (__uint_as_float(u[c]) - dv[e]);
+                    }
+                }
             }
             tc_fence_before();
-            if (it > 0 && !(ok = mbar_wait(&bars->ds_empty, (it - 1) & 1, g, 33))) break;
-            {
-                const uint32_t rowaddr = smem_u32(sDSb) + r * 128;
+            if (it > 0 && !mbar_wait(&bars->ds_empty, (it - 1) & 1, g, 33)) return false;
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint32_t a = pack_bf16x2(pv[8 * cc + 0], pv[8 * cc + 1]);
-                    const uint32_t b = pack_bf16x2(pv[8 * cc + 2], pv[8 * cc + 3]);
-                    const uint32_t c2 = pack_bf16x2(pv[8 * cc + 4], pv[8 * cc + 5]);
-                    const uint32_t d2 = pack_bf16x2(pv[8 * cc + 6], pv[8 * cc + 7]);
-                    st_shared_v4(rowaddr + ((cc ^ (r & 7)) << 4), a, b, c2, d2);
-                }
+            for (int cc = 0; cc < 8; ++cc) {
+                st_shared_v4(sDSrow + ((cc ^ (r & 7)) << 4), pack_bf16x2(pv[8 * cc + 0], pv[8 * cc + 1]),
+                             pack_bf16x2(pv[8 * cc + 2], pv[8 * cc + 3]),
+                             pack_bf16x2(pv[8 * cc + 4], pv[8 * cc + 5]),
+                             pack_bf16x2(pv[8 * cc + 6], pv[8 * cc + 7]));
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars->ds_full);
-            // ---- dQ_i readout (lane = query), staged for the bulk reduce
-            if (!(ok = mbar_wait_warp(&bars->dq_full, it & 1, g, 34))) break;
-            tc_fence_after();
+            return true;
+        };
+        // ---- dQr(it): dQ_i (lane = query) -> 128-B-swizzled fp32 staging, one
+        // 32-column box (16 KB) per 128 B of each row; the reducer adds it to
+        // the fp32 accumulator with TMA reduce-add.
+        auto phase_dQr = [&](int it) -> bool {
             constexpr int HC = D / 2;  // columns of dQ this warp reads
+            if (!mbar_wait_warp(&bars->dq_full, it & 1, g, 34)) return false;
+            tc_fence_after();
             uint32_t u[HC];
 #pragma unroll
             for (int c = 0; c < HC; c += 32)
@@ -417,19 +481,26 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             reg_fence<HC>(u);
             tc_fence_before();
             mbar_arrive(&bars->dq_empty);
-            if (it > 0 && !(ok = mbar_wait(&bars->dq_free, (it - 1) & 1, g, 35))) break;
-            {
-                float* rowp = sDQ + static_cast<size_t>(r) * D + HC * half;
+            if (it > 0 && !mbar_wait(&bars->dq_free, (it - 1) & 1, g, 35)) return false;
 #pragma unroll
-                for (int v = 0; v < HC / 4; ++v) {
-                    const int cc = (v + lane) % (HC / 4);  // rotate to spread banks
-                    reinterpret_cast<uint4*>(rowp)[cc] =
-                        make_uint4(u[4 * cc], u[4 * cc + 1], u[4 * cc + 2], u[4 * cc + 3]);
-                }
+            for (int b = 0; b < HC / 32; ++b) {
+                const uint32_t row = sDQ + (HC / 32 * half + b) * 16384 + r * 128;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+                    st_shared_v4(row + ((cc ^ (r & 7)) << 4), u[32 * b + 4 * cc],
+                                 u[32 * b + 4 * cc + 1], u[32 * b + 4 * cc + 2],
+                                 u[32 * b + 4 * cc + 3]);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars->dq_staged);
-        }
+            return true;
+        };
+
+        if (n_iter > 0) ok = phase_P(0) && phase_dS(0);
+        for (int it = 1; ok && it < n_iter; ++it)
+            ok = phase_P(it) && phase_dQr(it - 1) && phase_dS(it);
+        if (ok && n_iter > 0) ok = phase_dQr(n_iter - 1);
+
         // ---- dK, dV epilogue (lane = key)
         if (ok && mbar_wait_warp(&bars->dkdv_full, 0, g, 36)) {
             tc_fence_after();
@@ -502,10 +573,11 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         if (cudaGetLastError() != cudaSuccess) return false;
     }
     {
-        CUtensorMap mq, mk, mv, mdo;
+        CUtensorMap mq, mk, mv, mdo, mdq;
         const uint64_t depth = static_cast<uint64_t>(B) * H;
         if (!make_map_bf16_3d(&mq, Q, depth, N, D, 128) || !make_map_bf16_3d(&mk, K, depth, N, D, 128) ||
-            !make_map_bf16_3d(&mv, V, depth, N, D, 128) || !make_map_bf16_3d(&mdo, dO, depth, N, D, 128))
+            !make_map_bf16_3d(&mv, V, depth, N, D, 128) || !make_map_bf16_3d(&mdo, dO, depth, N, D, 128) ||
+            !make_map_f32_3d_sw128(&mdq, dQacc, depth, Npad, D))
             return false;
         BwdParams p;
         p.Dvec = Dvec;
@@ -521,7 +593,8 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         p.causal = causal ? 1 : 0;
         p.err = err;
         dim3 grid(Npad / 128, H, B);
-        fa_bwd_main_kernel<D><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+        fa_bwd_main_kernel<D><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
+                                                                                   mdq, p);
         if (cudaGetLastError() != cudaSuccess) return false;
     }
     {

@@ -40,10 +40,10 @@ constexpr int FWD_BM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int FWD_BN = 128;          // keys per block
 constexpr int FWD_THREADS = 384;     // 12 warps = 3 warpgroups
 // Registers: launched at 168/thread (384 x 168 = 64512); the control
-// warpgroup gives back down to 56 and each softmax warpgroup takes 224:
-// 2 x 128 x 224 + 128 x 56 = 64512.
-constexpr uint32_t FWD_REGS_SOFTMAX = 224;
-constexpr uint32_t FWD_REGS_CONTROL = 56;
+// warpgroup gives back down to 72 and each softmax warpgroup takes 216:
+// 2 x 128 x 216 + 128 x 72 = 64512.
+constexpr uint32_t FWD_REGS_SOFTMAX = 216;
+constexpr uint32_t FWD_REGS_CONTROL = 72;
 constexpr float FWD_RESCALE_TAU = 8.0f;  // log2 units: keep a stale row max while p <= 2^8
 
 template <int D>

@@ -90,7 +90,8 @@ __device__ __forceinline__ void guard_fail(const Guard& g, uint32_t code) {
 // Wait until the phase with the given parity has completed.  Returns false
 // (after recording `site`) on timeout or when another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Guard& g,
-                                          uint32_t site) {
+                                          uint32_t site,
+                                          uint64_t timeout_ns = FA_WAIT_TIMEOUT_NS) {
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
@@ -98,7 +99,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
         for (int i = 0; i < 32; ++i)
             if (mbar_test(bar, parity)) return true;
         if (*g.abort_flag) return false;
-        if (globaltimer() - t0 > FA_WAIT_TIMEOUT_NS) {
+        if (globaltimer() - t0 > timeout_ns) {
             guard_fail(g, DEV_TIMEOUT_BASE + site);
             return false;
         }
@@ -191,6 +192,17 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
+}
+
+// 3-D tiled shared -> global add-reduction (tensor map element type decides
+// the arithmetic, e.g. fp32 add), tracked by the bulk async-group.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* smem_src,
+                                                  int32_t x, int32_t y, int32_t z) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group"
+        " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+        : "memory");
 }
 
 // Contiguous global -> shared copy (16-byte aligned, size multiple of 16).
@@ -416,6 +428,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
                  : "memory");
+}
+
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t saddr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(saddr)
+                 : "memory");
+    return v;
 }
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
