@@ -49,12 +49,14 @@ constexpr float FWD_RESCALE_TAU = 8.0f;  // log2 units: keep a stale row max whi
 template <int D>
 struct FwdCfg {
     static constexpr int TILE_BYTES = FWD_BM * D * 2;  // one Q, K or V tile (bf16)
-    static constexpr int NSTAGE = (D == 128) ? 2 : 3;  // K/V ring depth
+    static constexpr int NK = 3;                       // K ring depth
+    static constexpr int NV = (D == 128) ? 2 : 3;      // V ring depth
+    static constexpr int PREFETCH = 2;                 // L2 prefetch distance beyond the rings
     static constexpr int CHUNKS = D / 64;              // 64-wide (128 B) TMA boxes per tile
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
-    static constexpr int OFF_V = OFF_K + NSTAGE * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_V + NSTAGE * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + NV * TILE_BYTES;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
@@ -77,7 +79,7 @@ struct FwdBars {
     uint64_t q_full;
     uint64_t k_full[3], k_empty[3];
     uint64_t v_full[3], v_empty[3];
-    uint64_t s_full[2], p_full[2], o_full[2];
+    uint64_t s_full[2], p_full[2][2], o_full[2];  // p_full[tile][key half]
 };
 
 template <int D>
@@ -120,15 +122,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         mbar_init(&bars->q_full, 1);
-        for (int s = 0; s < C::NSTAGE; ++s) {
+        for (int s = 0; s < C::NK; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
+        }
+        for (int s = 0; s < C::NV; ++s) {
             mbar_init(&bars->v_full[s], 1);
             mbar_init(&bars->v_empty[s], 1);
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars->s_full[t], 1);
-            mbar_init(&bars->p_full[t], 128);
+            mbar_init(&bars->p_full[t][0], 128);
+            mbar_init(&bars->p_full[t][1], 128);
             mbar_init(&bars->o_full[t], 1);
         }
         fence_barrier_init();
@@ -159,32 +164,41 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(smem + C::OFF_Q + t * C::TILE_BYTES + c * 16384, &mapQ,
                                 &bars->q_full, c * 64, q0 + t * FWD_BM, bh);
+            // K(j) and V(j) go to their own rings; L2 is asked for the tiles
+            // PREFETCH blocks beyond what the rings hold.
             int k_issued = 0, v_issued = 0;
             for (int j = 0; j < n_blocks; ++j) {
-                const int s = j % C::NSTAGE;
-                const uint32_t ph = (j / C::NSTAGE) & 1;
-                if (j >= C::NSTAGE && !mbar_wait(&bars->k_empty[s], ph ^ 1, g, 1)) break;
-                mbar_arrive_expect_tx(&bars->k_full[s], C::TILE_BYTES);
+                const int sk = j % C::NK, sv = j % C::NV;
+                if (j >= C::NK && !mbar_wait(&bars->k_empty[sk], ((j / C::NK) & 1) ^ 1, g, 1)) break;
+                mbar_arrive_expect_tx(&bars->k_full[sk], C::TILE_BYTES);
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
-                    tma_load_3d(smem + C::OFF_K + s * C::TILE_BYTES + c * 16384, &mapK,
-                                &bars->k_full[s], c * 64, j * FWD_BN, bh);
+                    tma_load_3d(smem + C::OFF_K + sk * C::TILE_BYTES + c * 16384, &mapK,
+                                &bars->k_full[sk], c * 64, j * FWD_BN, bh);
                 k_issued = j + 1;
-                if (j >= C::NSTAGE && !mbar_wait(&bars->v_empty[s], ph ^ 1, g, 2)) break;
-                mbar_arrive_expect_tx(&bars->v_full[s], C::TILE_BYTES);
+                const int jp = j + C::NK + C::PREFETCH - 1;
+                if (jp < n_blocks) {
+#pragma unroll
+                    for (int c = 0; c < C::CHUNKS; ++c) {
+                        tma_prefetch_l2_3d(&mapK, c * 64, jp * FWD_BN, bh);
+                        tma_prefetch_l2_3d(&mapV, c * 64, jp * FWD_BN, bh);
+                    }
+                }
+                if (j >= C::NV && !mbar_wait(&bars->v_empty[sv], ((j / C::NV) & 1) ^ 1, g, 2)) break;
+                mbar_arrive_expect_tx(&bars->v_full[sv], C::TILE_BYTES);
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
-                    tma_load_3d(smem + C::OFF_V + s * C::TILE_BYTES + c * 16384, &mapV,
-                                &bars->v_full[s], c * 64, j * FWD_BN, bh);
+                    tma_load_3d(smem + C::OFF_V + sv * C::TILE_BYTES + c * 16384, &mapV,
+                                &bars->v_full[sv], c * 64, j * FWD_BN, bh);
                 v_issued = j + 1;
             }
             // Never leave the CTA with copies still landing in its shared
             // memory: wait (bounded) for the last load issued into each slot.
             mbar_drain(&bars->q_full, 0);
-            for (int j = max(0, k_issued - C::NSTAGE); j < k_issued; ++j)
-                mbar_drain(&bars->k_full[j % C::NSTAGE], (j / C::NSTAGE) & 1);
-            for (int j = max(0, v_issued - C::NSTAGE); j < v_issued; ++j)
-                mbar_drain(&bars->v_full[j % C::NSTAGE], (j / C::NSTAGE) & 1);
+            for (int j = max(0, k_issued - C::NK); j < k_issued; ++j)
+                mbar_drain(&bars->k_full[j % C::NK], (j / C::NK) & 1);
+            for (int j = max(0, v_issued - C::NV); j < v_issued; ++j)
+                mbar_drain(&bars->v_full[j % C::NV], (j / C::NV) & 1);
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
@@ -208,10 +222,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     mma_ss(tS[t], a, b, idS, kk > 0);
                 }
             };
-            // O_t (+)= P_t V_j : P from TMEM (8 columns per k = 16), V MN-major.
-            auto issue_PV = [&](int t, int s, bool acc) {
+            // O_t (+)= P_t V_j for keys [64h, 64h + 64): P from TMEM (8 columns
+            // per k = 16), V MN-major.  The two halves are issued as soon as the
+            // softmax warps release each half of P.
+            auto issue_PV_half = [&](int t, int s, int h, bool acc) {
 #pragma unroll
-                for (int kk = 0; kk < FWD_BN / 16; ++kk) {
+                for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
                     const uint64_t b = sdesc_sw128(sV + s * C::TILE_BYTES + kk * 2048, 16384, 1024);
                     mma_ts(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
                 }
@@ -228,30 +244,40 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             }
             for (int j = 1; ok && j <= n_blocks; ++j) {
                 // Finish block j-1 (P.V) for both tiles, then start block j (S).
-                const int sp = (j - 1) % C::NSTAGE;
-                const uint32_t php = ((j - 1) / C::NSTAGE) & 1;
-                const int s = j % C::NSTAGE;
-                const uint32_t ph = (j / C::NSTAGE) & 1;
+                // Each wait sits right before the first MMA that needs it, and
+                // V(j-1)'s slot is released right after its last P.V.
+                const int sv = (j - 1) % C::NV;
+                const uint32_t phv = ((j - 1) / C::NV) & 1;
+                const int sk = j % C::NK;
+                const uint32_t phk = (j / C::NK) & 1;
                 const bool more = j < n_blocks;
-                if (more && !(ok = mbar_wait(&bars->k_full[s], ph, g, 5))) break;
-                if (!(ok = mbar_wait(&bars->v_full[sp], php, g, 6))) break;
+                bool k_ready = false;
+                if (!(ok = mbar_wait(&bars->v_full[sv], phv, g, 6))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     if (j - 1 < n_tile[t]) {
-                        if (!(ok = mbar_wait(&bars->p_full[t], (j - 1) & 1, g, 7 + t))) break;
+                        if (!(ok = mbar_wait(&bars->p_full[t][0], (j - 1) & 1, g, 7 + t))) break;
                         tc_fence_after();
-                        issue_PV(t, sp, j > 1);
+                        issue_PV_half(t, sv, 0, j > 1);
+                        if (!(ok = mbar_wait(&bars->p_full[t][1], (j - 1) & 1, g, 13 + t))) break;
+                        tc_fence_after();
+                        issue_PV_half(t, sv, 1, true);
                         if (j == n_tile[t]) tc_commit(&bars->o_full[t]);
                     }
+                    if (t == 1) tc_commit(&bars->v_empty[sv]);
                     if (more && j < n_tile[t]) {
-                        issue_S(t, s);
+                        if (!k_ready) {
+                            if (!(ok = mbar_wait(&bars->k_full[sk], phk, g, 5))) break;
+                            tc_fence_after();
+                            k_ready = true;
+                        }
+                        issue_S(t, sk);
                         tc_commit(&bars->s_full[t]);
                     }
                 }
                 if (!ok) break;
-                tc_commit(&bars->v_empty[sp]);
-                if (more) tc_commit(&bars->k_empty[s]);
+                if (more) tc_commit(&bars->k_empty[sk]);
             }
         }
     } else {
@@ -354,6 +380,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     ar[i % 4] = __fadd2_rn(ar[i % 4], unpack_bf16x2(pk[i]));
                 }
                 tmem_st32(tS + h * 32, pk);
+                // Release this half of P: the tensor core starts on keys
+                // [64h, 64h + 64) while the other half is still being computed.
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars->p_full[t][h]);
             }
             {
                 const float2 e = __fadd2_rn(__fadd2_rn(ae[0], ae[1]), __fadd2_rn(ae[2], ae[3]));
@@ -361,9 +392,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 l += e.x + e.y;
                 lr += r.x + r.y;
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full[t]);
         }
         // ------------------------------------------------------------ epilogue
         if (ok && mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t)) {
