@@ -69,6 +69,10 @@ struct BwdCfg {
     static constexpr bool DQ_ALIAS = (D == 128);  // dQ shares the dP^T columns
     static constexpr bool EARLY_S = (QS >= 2);    // issue S^T(i+1) before dK/dQ(i)
     static constexpr uint32_t T_DQ = DQ_ALIAS ? T_DPT : 256 + 2 * D;
+    // P^T: its own 64 columns when they exist (d = 64); over S^T otherwise,
+    // which needs both column halves of a lane read before either writes.
+    static constexpr bool P_ALIAS = (D == 128);
+    static constexpr uint32_t T_PT = P_ALIAS ? T_ST : 256 + 3 * D;
 };
 
 struct BwdBars {
@@ -293,7 +297,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             auto mma_dV = [&](int it) {  // dV += P^T dO   (P^T from TMEM)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + C::T_DV, tmem + C::T_ST + kk * 8,
+                    mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
                            sdesc_sw128(sdO(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
             };
             auto mma_dK_dQ = [&](int it) {  // dK += dS^T Q ; dQ = dS K
@@ -415,15 +419,17 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
                     if (key >= p.N || q >= p.N || q < qlim) pv[c] = 0.f;
                 }
             }
-            // Both column halves of these lanes must have read S^T before P^T
-            // (which overlaps it) is written.
-            mbar_arrive(&bars->pair[quarter]);
-            if (!mbar_wait_warp(&bars->pair[quarter], it & 1, g, 31)) return false;
+            if (C::P_ALIAS) {
+                // Both column halves of these lanes must have read S^T before
+                // P^T (which overlaps it) is written.
+                mbar_arrive(&bars->pair[quarter]);
+                if (!mbar_wait_warp(&bars->pair[quarter], it & 1, g, 31)) return false;
+            }
             {
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
-                tmem_st32(tmem_addr(tmem, lane_base, C::T_ST + 32 * half), pk);
+                tmem_st32(tmem_addr(tmem, lane_base, C::T_PT + 32 * half), pk);
             }
             tmem_st_wait();
             tc_fence_before();
