@@ -65,6 +65,17 @@ fa_status fa_forward(const void *Q, const void *K, const void *V, void *O, float
                      cudaStream_t stream);
 
 /*
+ * Grouped-query / multi-query attention ("FlashAttention-2" item 3 of the
+ * unite.ai page: grouped and multi-query attention).  Q and O have H heads;
+ * K and V have H_kv heads ([B, H_kv, N, d]); query head h of a batch uses
+ * K/V head h / (H / H_kv).  H_kv must divide H (H_kv = 1: multi-query;
+ * H_kv = H: identical to fa_forward).  FA_ERR_INVALID_ARG otherwise.
+ */
+fa_status fa_forward_gqa(const void *Q, const void *K, const void *V, void *O, float *LSE,
+                         int B, int H, int H_kv, int N, int d, float scale, int causal,
+                         cudaStream_t stream);
+
+/*
  * Device workspace fa_backward needs, in bytes (0 on invalid shapes).  It holds
  * D_i = <dO_i, O_i>, LSE in base-2 units and the fp32 dQ accumulator, each
  * padded to a multiple of 128 rows per head.
@@ -90,6 +101,18 @@ fa_status fa_backward(const void *Q, const void *K, const void *V, const void *O
                       void *workspace, size_t workspace_bytes,
                       int B, int H, int N, int d, float scale, int causal,
                       cudaStream_t stream);
+
+/*
+ * Backward of fa_forward_gqa: dQ is [B,H,N,d]; dK and dV are [B,H_kv,N,d],
+ * each the sum over the H / H_kv query heads that share the K/V head (summed
+ * in fp32 inside the kernel, deterministic).  Workspace as for fa_backward
+ * with H query heads: fa_backward_workspace_bytes(B, H, N, d).
+ */
+fa_status fa_backward_gqa(const void *Q, const void *K, const void *V, const void *O,
+                          const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
+                          void *workspace, size_t workspace_bytes,
+                          int B, int H, int H_kv, int N, int d, float scale, int causal,
+                          cudaStream_t stream);
 
 /*
  * Size of the device array fa_backward_noalloc uses as its workspace (64 MiB).

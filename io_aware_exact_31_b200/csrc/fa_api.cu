@@ -78,16 +78,23 @@ fa_status check_shape(int B, int H, int N, int d, float scale) {
     return FA_OK;
 }
 
+// H_kv: K/V heads per batch (H_kv divides H; H_kv == H is plain multi-head).
+fa_status check_heads(int H, int Hkv) {
+    if (Hkv < 1 || Hkv > H || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
 template <int D>
 fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const void* V, void* O,
-                         float* LSE, int B, int H, int N, float scale, int causal,
+                         float* LSE, int B, int H, int Hkv, int N, float scale, int causal,
                          cudaStream_t stream) {
     using C = FwdCfg<D>;
     CUtensorMap mq, mk, mv;
     const uint64_t depth = static_cast<uint64_t>(B) * H;
+    const uint64_t depth_kv = static_cast<uint64_t>(B) * Hkv;
     if (!make_map_bf16_3d(&mq, Q, depth, N, D, FWD_BM) ||
-        !make_map_bf16_3d(&mk, K, depth, N, D, FWD_BN) ||
-        !make_map_bf16_3d(&mv, V, depth, N, D, FWD_BN))
+        !make_map_bf16_3d(&mk, K, depth_kv, N, D, FWD_BN) ||
+        !make_map_bf16_3d(&mv, V, depth_kv, N, D, FWD_BN))
         return FA_ERR_CUDA;
     const int di = (D == 128) ? 1 : 0;
     if (!ds->fwd_attr[di]) {
@@ -105,6 +112,8 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     p.causal = causal ? 1 : 0;
     p.err = ds->err;
     p.n_heads = B * H;
+    p.H = H;
+    p.group = H / Hkv;
     p.n_pairs = (N + 2 * FWD_BM - 1) / (2 * FWD_BM);
     const long long n_ctas = static_cast<long long>(p.n_pairs) * p.n_heads;
     if (n_ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
@@ -145,17 +154,25 @@ using namespace fa;
 
 extern "C" {
 
-fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                     int H, int N, int d, float scale, int causal, cudaStream_t stream) {
+fa_status fa_forward_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                         int H, int H_kv, int N, int d, float scale, int causal,
+                         cudaStream_t stream) {
     if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
         return FA_ERR_INVALID_ARG;
     fa_status st = check_shape(B, H, N, d, scale);
     if (st != FA_OK) return st;
+    if ((st = check_heads(H, H_kv)) != FA_OK) return st;
     DeviceState* ds = current_device(&st);
     if (!ds) return st;
-    return d == 128 ? launch_forward<128>(ds, Q, K, V, O, LSE, B, H, N, scale, causal, stream)
-                    : launch_forward<64>(ds, Q, K, V, O, LSE, B, H, N, scale, causal, stream);
+    return d == 128
+               ? launch_forward<128>(ds, Q, K, V, O, LSE, B, H, H_kv, N, scale, causal, stream)
+               : launch_forward<64>(ds, Q, K, V, O, LSE, B, H, H_kv, N, scale, causal, stream);
+}
+
+fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int H, int N, int d, float scale, int causal, cudaStream_t stream) {
+    return fa_forward_gqa(Q, K, V, O, LSE, B, H, H, N, d, scale, causal, stream);
 }
 
 size_t fa_backward_workspace_bytes(int B, int H, int N, int d) {
@@ -163,10 +180,10 @@ size_t fa_backward_workspace_bytes(int B, int H, int N, int d) {
     return bwd_workspace_bytes(B, H, N, d);
 }
 
-fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                      const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
-                      size_t workspace_bytes, int B, int H, int N, int d, float scale,
-                      int causal, cudaStream_t stream) {
+fa_status fa_backward_gqa(const void* Q, const void* K, const void* V, const void* O,
+                          const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                          void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int N,
+                          int d, float scale, int causal, cudaStream_t stream) {
     if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace)
         return FA_ERR_INVALID_ARG;
     const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
@@ -174,6 +191,7 @@ fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O
         if (!aligned16(p)) return FA_ERR_INVALID_ARG;
     fa_status st = check_shape(B, H, N, d, scale);
     if (st != FA_OK) return st;
+    if ((st = check_heads(H, H_kv)) != FA_OK) return st;
     if (workspace_bytes < bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
     DeviceState* ds = current_device(&st);
     if (!ds) return st;
@@ -182,10 +200,18 @@ fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O
         if (!bwd_set_attributes(d)) return FA_ERR_CUDA;
         ds->bwd_attr[di] = true;
     }
-    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, N, d, scale, causal,
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, H_kv, N, d, scale, causal,
                       ds->err, stream)
                ? FA_OK
                : FA_ERR_CUDA;
+}
+
+fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                      const float* LSE, void* dQ, void* dK, void* dV, void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                      int causal, cudaStream_t stream) {
+    return fa_backward_gqa(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, B, H, H,
+                           N, d, scale, causal, stream);
 }
 
 fa_status fa_check_device_error(cudaStream_t stream, unsigned int* site) {
@@ -294,7 +320,7 @@ extern "C" fa_status fa_backward_noalloc(const void* Q, const void* K, const voi
     // Same three kernels as fa_backward; the preprocess kernel rewrites every
     // byte of the scratch the later kernels read (D, LSE and the zeroed fp32
     // dQ accumulator), so what an earlier call left there does not matter.
-    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, scratch, B, H, N, d, scale, causal,
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, scratch, B, H, H, N, d, scale, causal,
                       ds->err, stream)
                ? FA_OK
                : FA_ERR_CUDA;

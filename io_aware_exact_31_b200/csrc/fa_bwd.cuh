@@ -37,9 +37,9 @@ constexpr int BWD_BM = 128;  // queries per block
 constexpr int BWD_BN = 128;  // keys per CTA
 constexpr int BWD_THREADS = 384;  // 3 warpgroups
 // Registers: launched at 168 (384 x 168 = 64512); the control warpgroup drops
-// to 72 and the two compute warpgroups rise to 216: 256 x 216 + 128 x 72.
-constexpr uint32_t BWD_REGS_COMPUTE = 216;
-constexpr uint32_t BWD_REGS_CONTROL = 72;
+// to 88 and the two compute warpgroups rise to 208: 256 x 208 + 128 x 88.
+constexpr uint32_t BWD_REGS_COMPUTE = 208;
+constexpr uint32_t BWD_REGS_CONTROL = 88;
 
 inline size_t round_up_128(int n) { return (static_cast<size_t>(n) + 127) / 128 * 128; }
 
@@ -90,6 +90,7 @@ struct BwdParams {
     __nv_bfloat16* dK;
     __nv_bfloat16* dV;
     int N, Npad, n_q_blocks;
+    int H, group;        // query heads per batch; query heads per K/V head
     float scale, scale_log2;
     int causal;
     uint32_t* err;
@@ -191,11 +192,18 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     const Guard g{abort_flag, p.err};
 
     const uint32_t warp = warp_id(), lane = lane_id();
-    const int bh = blockIdx.z * gridDim.y + blockIdx.y;
+    // CTA = (key block, K/V head).  With grouped-query attention the CTA walks
+    // every query head of its group, so dK/dV sum over the group in TMEM.
+    const int bkv = blockIdx.z * gridDim.y + blockIdx.y;  // K/V head (b * H_kv + h_kv)
+    const int bq0 = blockIdx.z * p.H + blockIdx.y * p.group;  // first query head of the group
     const int kb = blockIdx.x;  // key block; causal: block 0 has the most work and starts first
     const int k0 = kb * BWD_BN;
     const int i_begin = p.causal ? kb : 0;  // first query block that sees this key block
-    const int n_iter = p.n_q_blocks - i_begin;
+    const int nq = p.n_q_blocks - i_begin;  // query blocks per query head
+    const int n_iter = nq * p.group;
+    // iteration it -> (query head, query block)
+    auto q_head = [&](int it) { return bq0 + it / nq; };
+    auto q_block0 = [&](int it) { return (i_begin + it % nq) * BWD_BM; };
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -239,14 +247,14 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
 #pragma unroll
             for (int c = 0; c < C::CHUNKS; ++c) {
-                tma_load_3d(smem + C::OFF_K + c * 16384, &mapK, &bars->kv_full, c * 64, k0, bh);
-                tma_load_3d(smem + C::OFF_V + c * 16384, &mapV, &bars->kv_full, c * 64, k0, bh);
+                tma_load_3d(smem + C::OFF_K + c * 16384, &mapK, &bars->kv_full, c * 64, k0, bkv);
+                tma_load_3d(smem + C::OFF_V + c * 16384, &mapV, &bars->kv_full, c * 64, k0, bkv);
             }
             int issued = 0;
             for (int it = 0; it < n_iter; ++it) {
                 const int s = it % C::QS;
                 const uint32_t ph = (it / C::QS) & 1;
-                const int q0 = (i_begin + it) * BWD_BM;
+                const int q0 = q_block0(it), bh = q_head(it);
                 if (it >= C::QS && !mbar_wait(&bars->q_empty[s], ph ^ 1, g, 21)) break;
                 mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::TILE + 1024);
 #pragma unroll
@@ -357,7 +365,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             tma_prefetch_desc(&mapdQacc);
             for (int it = 0; it < n_iter; ++it) {
                 if (!mbar_wait(&bars->dq_staged, it & 1, g, 28)) break;
-                const int q0 = (i_begin + it) * BWD_BM;
+                const int q0 = q_block0(it), bh = q_head(it);
 #pragma unroll
                 for (int b = 0; b < D / 32; ++b)
                     tma_reduce_add_3d(&mapdQacc, smem + C::OFF_DQ + b * 16384, b * 32, q0, bh);
@@ -384,7 +392,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         auto phase_P = [&](int it) -> bool {
             const int s = it % C::QS;
             const uint32_t ph = (it / C::QS) & 1;
-            const int q0 = (i_begin + it) * BWD_BM;
+            const int q0 = q_block0(it);
             const int qh = q0 + 64 * half;  // first query of this warp's columns
             if (!mbar_wait(&bars->q_full[s], ph, g, 29)) return false;
             if (!mbar_wait_warp(&bars->s_full, it & 1, g, 30)) return false;
@@ -512,7 +520,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             tc_fence_after();
             constexpr int HC = D / 2;
             const bool valid = key < p.N;
-            const size_t off = (static_cast<size_t>(bh) * p.N + (valid ? key : 0)) * D + HC * half;
+            const size_t off = (static_cast<size_t>(bkv) * p.N + (valid ? key : 0)) * D + HC * half;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const uint32_t col = (which == 0 ? C::T_DV : C::T_DK) + HC * half;
@@ -564,7 +572,7 @@ inline bool bwd_set_attributes(int d) {
 template <int D>
 bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                   const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
-                  int N, float scale, int causal, uint32_t* err, cudaStream_t stream) {
+                  int Hkv, int N, float scale, int causal, uint32_t* err, cudaStream_t stream) {
     const int Npad = static_cast<int>(round_up_128(N));
     const long long rows_pad = static_cast<long long>(B) * H * Npad;
     float* Dvec = static_cast<float*>(workspace);
@@ -581,8 +589,9 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
     {
         CUtensorMap mq, mk, mv, mdo, mdq;
         const uint64_t depth = static_cast<uint64_t>(B) * H;
-        if (!make_map_bf16_3d(&mq, Q, depth, N, D, 128) || !make_map_bf16_3d(&mk, K, depth, N, D, 128) ||
-            !make_map_bf16_3d(&mv, V, depth, N, D, 128) || !make_map_bf16_3d(&mdo, dO, depth, N, D, 128) ||
+        const uint64_t depth_kv = static_cast<uint64_t>(B) * Hkv;
+        if (!make_map_bf16_3d(&mq, Q, depth, N, D, 128) || !make_map_bf16_3d(&mk, K, depth_kv, N, D, 128) ||
+            !make_map_bf16_3d(&mv, V, depth_kv, N, D, 128) || !make_map_bf16_3d(&mdo, dO, depth, N, D, 128) ||
             !make_map_f32_3d_sw128(&mdq, dQacc, depth, Npad, D))
             return false;
         BwdParams p;
@@ -594,11 +603,13 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         p.N = N;
         p.Npad = Npad;
         p.n_q_blocks = Npad / 128;
+        p.H = H;
+        p.group = H / Hkv;
         p.scale = scale;
         p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
         p.causal = causal ? 1 : 0;
         p.err = err;
-        dim3 grid(Npad / 128, H, B);
+        dim3 grid(Npad / 128, Hkv, B);
         fa_bwd_main_kernel<D><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
                                                                                    mdq, p);
         if (cudaGetLastError() != cudaSuccess) return false;
@@ -615,11 +626,12 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
 
 inline bool bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                        const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
-                       int N, int d, float scale, int causal, uint32_t* err, cudaStream_t stream) {
-    return d == 128 ? bwd_launch_t<128>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, N, scale,
-                                        causal, err, stream)
-                    : bwd_launch_t<64>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, N, scale,
-                                       causal, err, stream);
+                       int Hkv, int N, int d, float scale, int causal, uint32_t* err,
+                       cudaStream_t stream) {
+    return d == 128 ? bwd_launch_t<128>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N,
+                                        scale, causal, err, stream)
+                    : bwd_launch_t<64>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N,
+                                       scale, causal, err, stream);
 }
 
 }  // namespace fa

@@ -69,7 +69,9 @@ struct FwdParams {
     int n_kv_blocks;    // ceil(N / 128)
     float scale_log2;   // scale * log2(e)
     int causal;
-    int n_heads;        // B * H
+    int n_heads;        // B * H (query heads)
+    int H;              // query heads per batch
+    int group;          // query heads per K/V head (H / H_kv; 1 = plain multi-head)
     int n_pairs;        // ceil(N / 256)
     uint32_t* err;      // device error word
 };
@@ -109,6 +111,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         bh = blockIdx.x / p.n_pairs;
         pair = blockIdx.x % p.n_pairs;
     }
+    // K/V head of this query head (grouped-query attention; = bh when group = 1).
+    const int bkv = (bh / p.H) * (p.H / p.group) + (bh % p.H) / p.group;
     const int q0 = pair * 2 * FWD_BM;
     // Key blocks each tile needs: causal tiles stop at their diagonal block.
     int n_tile[2];
@@ -174,14 +178,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(smem + C::OFF_K + sk * C::TILE_BYTES + c * 16384, &mapK,
-                                &bars->k_full[sk], c * 64, j * FWD_BN, bh);
+                                &bars->k_full[sk], c * 64, j * FWD_BN, bkv);
                 k_issued = j + 1;
                 const int jp = j + C::NK + C::PREFETCH - 1;
                 if (jp < n_blocks) {
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) {
-                        tma_prefetch_l2_3d(&mapK, c * 64, jp * FWD_BN, bh);
-                        tma_prefetch_l2_3d(&mapV, c * 64, jp * FWD_BN, bh);
+                        tma_prefetch_l2_3d(&mapK, c * 64, jp * FWD_BN, bkv);
+                        tma_prefetch_l2_3d(&mapV, c * 64, jp * FWD_BN, bkv);
                     }
                 }
                 if (j >= C::NV && !mbar_wait(&bars->v_empty[sv], ((j / C::NV) & 1) ^ 1, g, 2)) break;
@@ -189,7 +193,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(smem + C::OFF_V + sv * C::TILE_BYTES + c * 16384, &mapV,
-                                &bars->v_full[sv], c * 64, j * FWD_BN, bh);
+                                &bars->v_full[sv], c * 64, j * FWD_BN, bkv);
                 v_issued = j + 1;
             }
             // Never leave the CTA with copies still landing in its shared

@@ -51,13 +51,18 @@ def load(path: str | None = None):
                                                   vp, i64, vp, vp]
     lib.oracle_attention_backward.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, dbl, ip,
                                               vp, vp, vp]
+    lib.oracle_attention_forward_gqa.argtypes = [vp, vp, vp, ip, i64, i64, i64, i64, i64, dbl, ip,
+                                                 vp, vp]
+    lib.oracle_attention_backward_gqa.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, i64, dbl,
+                                                  ip, vp, vp, vp]
     lib.oracle_softmax_partial.argtypes = [vp, i64, vp, i64, vp, vp, vp]
     lib.oracle_softmax_merge.argtypes = [dbl, dbl, vp, dbl, dbl, vp, i64, vp, vp, vp]
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_num_threads.argtypes = [ip]
     for name in ("oracle_attention_forward", "oracle_attention_forward_rows",
                  "oracle_attention_backward", "oracle_softmax_partial",
-                 "oracle_softmax_merge"):
+                 "oracle_softmax_merge", "oracle_attention_forward_gqa",
+                 "oracle_attention_backward_gqa"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -127,6 +132,39 @@ def attention_backward(Q, K, V, dO, scale: float, causal: bool, lib=None):
                                          float(scale), int(bool(causal)),
                                          _ptr(dQ), _ptr(dK), _ptr(dV)),
            "oracle_attention_backward")
+    return dQ, dK, dV
+
+
+def attention_forward_gqa(Q, K, V, scale: float, causal: bool, lib=None):
+    """Grouped-query forward: Q [B,H,N,d], K/V [B,Hkv,N,d] -> O [B,H,N,d], LSE [B,H,N]."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv) = _as_input(Q), _as_input(K), _as_input(V)
+    assert dt == dk == dv and K.shape == V.shape and Q.ndim == 4
+    B, H, N, d = Q.shape
+    Hkv = K.shape[1]
+    O = np.empty((B, H, N, d), np.float64)
+    LSE = np.empty((B, H, N), np.float64)
+    _check(lib.oracle_attention_forward_gqa(_ptr(Q), _ptr(K), _ptr(V), dt, B, H, Hkv, N, d,
+                                            float(scale), int(bool(causal)), _ptr(O), _ptr(LSE)),
+           "oracle_attention_forward_gqa")
+    return O, LSE
+
+
+def attention_backward_gqa(Q, K, V, dO, scale: float, causal: bool, lib=None):
+    """Grouped-query backward: dQ [B,H,N,d]; dK, dV [B,Hkv,N,d] (sums over each group)."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv), (dO, dd) = (_as_input(Q), _as_input(K), _as_input(V),
+                                           _as_input(dO))
+    assert dt == dk == dv == dd and K.shape == V.shape and Q.shape == dO.shape
+    B, H, N, d = Q.shape
+    Hkv = K.shape[1]
+    dQ = np.empty((B, H, N, d), np.float64)
+    dK = np.empty((B, Hkv, N, d), np.float64)
+    dV = np.empty_like(dK)
+    _check(lib.oracle_attention_backward_gqa(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), dt, B, H, Hkv,
+                                             N, d, float(scale), int(bool(causal)),
+                                             _ptr(dQ), _ptr(dK), _ptr(dV)),
+           "oracle_attention_backward_gqa")
     return dQ, dK, dV
 
 

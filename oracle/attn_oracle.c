@@ -36,6 +36,12 @@
  * (dtype ORACLE_BF16, widened exactly to double on load).  Layout of every
  * tensor: contiguous [B, H, N, d] (d fastest); LSE is [B, H, N].
  *
+ *   [GQA]   same unite.ai page, "FlashAttention-2" item 3: grouped-query and
+ *           multi-query attention.  Reading: H query heads share H_kv key/
+ *           value heads (H_kv divides H); query head h of a batch attends
+ *           with key/value head h / (H / H_kv).  The *_gqa functions take
+ *           K, V as [B, H_kv, N, d]; with H_kv = H they are [STD] per head.
+ *
  * Every function returns 0 on success, -1 on a bad argument, -2 if memory
  * could not be allocated.
  */
@@ -67,8 +73,15 @@ static int bad_shape(int64_t B, int64_t H, int64_t N, int64_t d, int dtype)
            (dtype != ORACLE_F64 && dtype != ORACLE_BF16);
 }
 
+/* [GQA]: key/value head of query head bh = b * H + h. */
+static int64_t kv_head(int64_t bh, int64_t H, int64_t Hkv)
+{
+    return (bh / H) * Hkv + (bh % H) / (H / Hkv);
+}
+
 /*
- * One output row of [STD] for query i of head bh:
+ * One output row of [STD] for query i (queries of this head start at element
+ * q_base, its keys and values at kv_base):
  *   s_j   = scale * <q_i, k_j>           (s_j = -inf if causal and j > i)
  *   m     = max_j s_j                    ([SAFE])
  *   LSE_i = m + ln sum_j exp(s_j - m)
@@ -77,11 +90,10 @@ static int bad_shape(int64_t B, int64_t H, int64_t N, int64_t d, int dtype)
  * s is caller-provided scratch of N doubles.
  */
 static void attention_row(const void *Q, const void *K, const void *V, int dtype,
-                          int64_t N, int64_t d, int64_t bh, int64_t i,
+                          int64_t N, int64_t d, int64_t q_base, int64_t kv_base, int64_t i,
                           double scale, int causal, double *s,
                           double *o_row, double *lse)
 {
-    const int64_t base = bh * N * d;
     for (int64_t j = 0; j < N; ++j) {
         if (causal && j > i) {
             s[j] = -INFINITY;
@@ -89,7 +101,7 @@ static void attention_row(const void *Q, const void *K, const void *V, int dtype
         }
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c)
-            acc += ld(Q, base + i * d + c, dtype) * ld(K, base + j * d + c, dtype);
+            acc += ld(Q, q_base + i * d + c, dtype) * ld(K, kv_base + j * d + c, dtype);
         s[j] = scale * acc;
     }
     double m = -INFINITY;
@@ -108,16 +120,18 @@ static void attention_row(const void *Q, const void *K, const void *V, int dtype
         if (p == 0.0)
             continue;
         for (int64_t c = 0; c < d; ++c)
-            o_row[c] += p * ld(V, base + j * d + c, dtype);
+            o_row[c] += p * ld(V, kv_base + j * d + c, dtype);
     }
 }
 
-/* Full forward: O [B,H,N,d] and LSE [B,H,N], both double. */
-int oracle_attention_forward(const void *Q, const void *K, const void *V, int dtype,
-                             int64_t B, int64_t H, int64_t N, int64_t d,
-                             double scale, int causal, double *O, double *LSE)
+/* Full forward with [GQA] heads: O [B,H,N,d] and LSE [B,H,N], both double;
+ * K, V are [B,Hkv,N,d]. */
+int oracle_attention_forward_gqa(const void *Q, const void *K, const void *V, int dtype,
+                                 int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                 double scale, int causal, double *O, double *LSE)
 {
-    if (!Q || !K || !V || !O || !LSE || bad_shape(B, H, N, d, dtype))
+    if (!Q || !K || !V || !O || !LSE || bad_shape(B, H, N, d, dtype) ||
+        Hkv < 1 || Hkv > H || H % Hkv != 0)
         return -1;
     const int64_t rows = B * H * N;
     int failed = 0;
@@ -133,12 +147,20 @@ int oracle_attention_forward(const void *Q, const void *K, const void *V, int dt
             if (!s)
                 continue;
             const int64_t bh = r / N, i = r % N;
-            attention_row(Q, K, V, dtype, N, d, bh, i, scale, causal, s,
-                          O + r * d, LSE + r);
+            attention_row(Q, K, V, dtype, N, d, bh * N * d, kv_head(bh, H, Hkv) * N * d, i,
+                          scale, causal, s, O + r * d, LSE + r);
         }
         free(s);
     }
     return failed ? -2 : 0;
+}
+
+/* Full forward, one key/value head per query head. */
+int oracle_attention_forward(const void *Q, const void *K, const void *V, int dtype,
+                             int64_t B, int64_t H, int64_t N, int64_t d,
+                             double scale, int causal, double *O, double *LSE)
+{
+    return oracle_attention_forward_gqa(Q, K, V, dtype, B, H, H, N, d, scale, causal, O, LSE);
 }
 
 /*
@@ -172,7 +194,7 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
             if (!s)
                 continue;
             const int64_t bh = rows[k] / N, i = rows[k] % N;
-            attention_row(Q, K, V, dtype, N, d, bh, i, scale, causal, s,
+            attention_row(Q, K, V, dtype, N, d, bh * N * d, bh * N * d, i, scale, causal, s,
                           O_rows + k * d, LSE_rows + k);
         }
         free(s);
@@ -181,7 +203,8 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
 }
 
 /*
- * Exact gradient of [STD] for upstream gradient dO, one head at a time,
+ * Exact gradient of [STD] (with [GQA] heads) for upstream gradient dO, one
+ * query head at a time,
  * with the full N x N matrices P, dP and dS materialised ([RECOMP] says only
  * that the fast path recomputes instead of storing; the oracle stores).
  *   P_ij  = softmax_j(s_ij)                  (row i, masked keys give 0)
@@ -191,13 +214,17 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
  *   dS_ij = P_ij (dP_ij - D_i)
  *   dQ_i  = scale sum_j dS_ij k_j
  *   dK_j  = scale sum_i dS_ij q_i
- * Outputs dQ, dK, dV are double [B,H,N,d].
+ * With [GQA] heads the key/value gradients of a key/value head are the sums
+ * of these over the query heads that share it.  dQ is double [B,H,N,d];
+ * dK, dV are double [B,Hkv,N,d].
  */
-int oracle_attention_backward(const void *Q, const void *K, const void *V, const void *dO,
-                              int dtype, int64_t B, int64_t H, int64_t N, int64_t d,
-                              double scale, int causal, double *dQ, double *dK, double *dV)
+int oracle_attention_backward_gqa(const void *Q, const void *K, const void *V, const void *dO,
+                                  int dtype, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                                  int64_t d, double scale, int causal,
+                                  double *dQ, double *dK, double *dV)
 {
-    if (!Q || !K || !V || !dO || !dQ || !dK || !dV || bad_shape(B, H, N, d, dtype))
+    if (!Q || !K || !V || !dO || !dQ || !dK || !dV || bad_shape(B, H, N, d, dtype) ||
+        Hkv < 1 || Hkv > H || H % Hkv != 0)
         return -1;
     double *P = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
     double *dS = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
@@ -206,8 +233,13 @@ int oracle_attention_backward(const void *Q, const void *K, const void *V, const
         free(dS);
         return -2;
     }
+    for (int64_t e = 0; e < B * Hkv * N * d; ++e) {
+        dK[e] = 0.0;
+        dV[e] = 0.0;
+    }
     for (int64_t bh = 0; bh < B * H; ++bh) {
-        const int64_t base = bh * N * d;
+        const int64_t base = bh * N * d;                        /* Q, dO, dQ */
+        const int64_t kv_base = kv_head(bh, H, Hkv) * N * d;    /* K, V, dK, dV */
         /* P row by row, exactly as the forward defines it. */
 #pragma omp parallel for schedule(dynamic, 8)
         for (int64_t i = 0; i < N; ++i) {
@@ -219,7 +251,7 @@ int oracle_attention_backward(const void *Q, const void *K, const void *V, const
                 }
                 double acc = 0.0;
                 for (int64_t c = 0; c < d; ++c)
-                    acc += ld(Q, base + i * d + c, dtype) * ld(K, base + j * d + c, dtype);
+                    acc += ld(Q, base + i * d + c, dtype) * ld(K, kv_base + j * d + c, dtype);
                 s[j] = scale * acc;
             }
             double m = -INFINITY;
@@ -240,7 +272,7 @@ int oracle_attention_backward(const void *Q, const void *K, const void *V, const
             for (int64_t j = 0; j < N; ++j) {
                 double acc = 0.0;
                 for (int64_t c = 0; c < d; ++c)
-                    acc += ld(dO, base + i * d + c, dtype) * ld(V, base + j * d + c, dtype);
+                    acc += ld(dO, base + i * d + c, dtype) * ld(V, kv_base + j * d + c, dtype);
                 ds[j] = acc; /* dP_ij */
             }
             double D = 0.0;
@@ -255,7 +287,7 @@ int oracle_attention_backward(const void *Q, const void *K, const void *V, const
             for (int64_t c = 0; c < d; ++c) {
                 double acc = 0.0;
                 for (int64_t j = 0; j < N; ++j)
-                    acc += dS[i * N + j] * ld(K, base + j * d + c, dtype);
+                    acc += dS[i * N + j] * ld(K, kv_base + j * d + c, dtype);
                 dQ[base + i * d + c] = scale * acc;
             }
         }
@@ -268,14 +300,23 @@ int oracle_attention_backward(const void *Q, const void *K, const void *V, const
                     acc_k += dS[i * N + j] * ld(Q, base + i * d + c, dtype);
                     acc_v += P[i * N + j] * ld(dO, base + i * d + c, dtype);
                 }
-                dK[base + j * d + c] = scale * acc_k;
-                dV[base + j * d + c] = acc_v;
+                dK[kv_base + j * d + c] += scale * acc_k;
+                dV[kv_base + j * d + c] += acc_v;
             }
         }
     }
     free(P);
     free(dS);
     return 0;
+}
+
+/* Backward with one key/value head per query head. */
+int oracle_attention_backward(const void *Q, const void *K, const void *V, const void *dO,
+                              int dtype, int64_t B, int64_t H, int64_t N, int64_t d,
+                              double scale, int causal, double *dQ, double *dK, double *dV)
+{
+    return oracle_attention_backward_gqa(Q, K, V, dO, dtype, B, H, H, N, d, scale, causal,
+                                         dQ, dK, dV);
 }
 
 /*

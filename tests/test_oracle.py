@@ -363,6 +363,49 @@ def pin_backward_single_key(lib):
     _close(dK, np.zeros_like(dK))
 
 
+# ----------------------------------------------------------------------------
+# Grouped-query attention pins (unite.ai page, "FlashAttention-2" item 3)
+# ----------------------------------------------------------------------------
+
+def pin_gqa_forward_vs_torch(lib):
+    """Library special case: torch SDPA (fp64) with enable_gqa; and Hkv = H is
+    plain multi-head attention."""
+    r = _rng(21)
+    for (B, H, Hkv, N, d, causal) in [(2, 6, 2, 11, 8, False), (1, 4, 1, 9, 4, True),
+                                      (1, 4, 4, 7, 4, True)]:
+        Q = r.standard_normal((B, H, N, d))
+        K, V = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+        O, LSE = oracle.attention_forward_gqa(Q, K, V, 0.4, causal, lib=lib)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            *(torch.from_numpy(x) for x in (Q, K, V)), is_causal=causal, scale=0.4,
+            enable_gqa=True)
+        _close(O, ref.numpy())
+        Kr = np.repeat(K, H // Hkv, axis=1)
+        s = 0.4 * torch.from_numpy(Q) @ torch.from_numpy(Kr).transpose(-1, -2)
+        if causal:
+            s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+        _close(LSE, torch.logsumexp(s, dim=-1).numpy())
+
+
+def pin_gqa_backward_vs_autograd(lib):
+    """torch.autograd (fp64) through K/V repeated to every query head: the
+    gradient of a shared K/V head sums over its group."""
+    r = _rng(22)
+    for (B, H, Hkv, N, d, causal) in [(1, 6, 2, 9, 4, True), (2, 4, 1, 7, 8, False)]:
+        Q, dO = (r.standard_normal((B, H, N, d)) for _ in range(2))
+        K, V = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+        G = H // Hkv
+        s = 0.5 * tq @ tk.repeat_interleave(G, dim=1).transpose(-1, -2)
+        if causal:
+            s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+        (torch.softmax(s, dim=-1) @ tv.repeat_interleave(G, dim=1)).backward(torch.from_numpy(dO))
+        dQ, dK, dV = oracle.attention_backward_gqa(Q, K, V, dO, 0.5, causal, lib=lib)
+        _close(dQ, tq.grad.numpy())
+        _close(dK, tk.grad.numpy())
+        _close(dV, tv.grad.numpy())
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -412,8 +455,12 @@ MUTANTS = {
     "causal_flipped": ("if (causal && j > i)", "if (causal && j < i)", 0),
     "lse_missing_max": ("*lse = m + log(sum);", "*lse = log(sum);", 0),
     "no_normalisation": ("const double p = s[j] / sum;", "const double p = s[j];", 0),
-    "wrong_value_row": ("o_row[c] += p * ld(V, base + j * d + c, dtype);",
-                        "o_row[c] += p * ld(V, base + i * d + c, dtype);", 0),
+    "wrong_value_row": ("o_row[c] += p * ld(V, kv_base + j * d + c, dtype);",
+                        "o_row[c] += p * ld(V, kv_base + i * d + c, dtype);", 0),
+    "gqa_interleaved_heads": ("return (bh / H) * Hkv + (bh % H) / (H / Hkv);",
+                              "return (bh / H) * Hkv + (bh % H) % Hkv;", 0),
+    "gqa_dK_overwrites": ("dK[kv_base + j * d + c] += scale * acc_k;",
+                          "dK[kv_base + j * d + c] = scale * acc_k;", 0),
     "exp_sign": ("s[j] = exp(s[j] - m); /* exp(-inf)", "s[j] = exp(m - s[j]); /* exp(-inf)", 0),
     "bwd_drop_scale_in_scores": ("s[j] = scale * acc;", "s[j] = acc;", 1),
     "bwd_drop_D": ("ds[j] = P[i * N + j] * (ds[j] - D);", "ds[j] = P[i * N + j] * ds[j];", 0),
