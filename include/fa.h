@@ -76,6 +76,19 @@ fa_status fa_forward_gqa(const void *Q, const void *K, const void *V, void *O, f
                          cudaStream_t stream);
 
 /*
+ * Padded batches (the padding mask of downcodes.com "triton transformer",
+ * BERT example).  seqlens: DEVICE pointer to B int32 values, seqlens[b] in
+ * 0..N real tokens of batch b (values outside are clamped), or NULL (all N
+ * real, identical to fa_forward_gqa).  Tokens >= seqlens[b] are padding: as
+ * keys they are masked for every query; as queries their O rows and LSE are
+ * written as 0.  Key blocks entirely in the padding are not read.  Otherwise
+ * as fa_forward_gqa (K/V with H_kv heads).
+ */
+fa_status fa_forward_varlen(const void *Q, const void *K, const void *V, void *O, float *LSE,
+                            const int *seqlens, int B, int H, int H_kv, int N, int d,
+                            float scale, int causal, cudaStream_t stream);
+
+/*
  * Device workspace fa_backward needs, in bytes (0 on invalid shapes).  It holds
  * D_i = <dO_i, O_i>, LSE in base-2 units and the fp32 dQ accumulator, each
  * padded to a multiple of 128 rows per head.
@@ -113,6 +126,16 @@ fa_status fa_backward_gqa(const void *Q, const void *K, const void *V, const voi
                           void *workspace, size_t workspace_bytes,
                           int B, int H, int H_kv, int N, int d, float scale, int causal,
                           cudaStream_t stream);
+
+/*
+ * Backward of fa_forward_varlen (same seqlens): padding query rows contribute
+ * nothing and every gradient row of a padding token is written as 0.
+ */
+fa_status fa_backward_varlen(const void *Q, const void *K, const void *V, const void *O,
+                             const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
+                             void *workspace, size_t workspace_bytes, const int *seqlens,
+                             int B, int H, int H_kv, int N, int d, float scale, int causal,
+                             cudaStream_t stream);
 
 /*
  * Size of the device array fa_backward_noalloc uses as its workspace (64 MiB).

@@ -18,9 +18,9 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 
 # Every entry point include/fa.h declares.
-EXPORTS = ("fa_forward", "fa_forward_gqa", "fa_backward_workspace_bytes", "fa_backward",
-           "fa_backward_gqa", "fa_backward_noalloc", "fa_check_device_error",
-           "fa_selftest_bounded_wait", "fa_status_str", "fa_version")
+EXPORTS = ("fa_forward", "fa_forward_gqa", "fa_forward_varlen", "fa_backward_workspace_bytes",
+           "fa_backward", "fa_backward_gqa", "fa_backward_varlen", "fa_backward_noalloc",
+           "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_str", "fa_version")
 
 # Size of the library's built-in workspace used by fa_backward_noalloc.
 NOALLOC_MAX_SCRATCH_BYTES = 64 * 1024 * 1024
@@ -56,6 +56,11 @@ def load_library(path: str | None = None):
     lib.fa_backward_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f,
                                     i, vp]
     lib.fa_backward_gqa.restype = i
+    lib.fa_forward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.fa_forward_varlen.restype = i
+    lib.fa_backward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, i, i, i, i,
+                                       i, f, i, vp]
+    lib.fa_backward_varlen.restype = i
     lib.fa_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_backward_noalloc.restype = i
     lib.fa_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -111,11 +116,21 @@ def backward_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(load_library().fa_backward_workspace_bytes(B, H, N, d))
 
 
+def _seqlens_ptr(seqlens, B, device):
+    if seqlens is None:
+        return None, None
+    t = seqlens.to(device=device, dtype=torch.int32).contiguous()
+    if t.shape != (B,):
+        raise ValueError("seqlens must have shape [B]")
+    return t, t.data_ptr()
+
+
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
             scale: float | None = None, out: torch.Tensor | None = None,
-            lse: torch.Tensor | None = None, stream=None):
+            lse: torch.Tensor | None = None, stream=None, seqlens: torch.Tensor | None = None):
     """O, LSE = softmax(scale Q K^T [+causal]) V and its per-row logsumexp.
-    K and V may have fewer heads than Q (grouped-/multi-query attention)."""
+    K and V may have fewer heads than Q (grouped-/multi-query attention);
+    seqlens [B] marks tokens >= seqlens[b] of batch b as padding."""
     B, H, N, d, Hkv = _check_kv_heads(q, k, v)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
@@ -123,16 +138,18 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fa
     _check_qkv(q, o)
     if l.dtype != torch.float32 or not l.is_contiguous() or tuple(l.shape) != (B, H, N):
         raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
-    st = load_library().fa_forward_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                       l.data_ptr(), B, H, Hkv, N, d, scale, int(bool(causal)),
-                                       _stream_handle(stream))
+    keep, sl = _seqlens_ptr(seqlens, B, q.device)
+    st = load_library().fa_forward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                          l.data_ptr(), sl, B, H, Hkv, N, d, scale,
+                                          int(bool(causal)), _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_forward")
     return o, l
 
 
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
-             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, stream=None):
+             dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, stream=None,
+             seqlens: torch.Tensor | None = None):
     """dQ, dK, dV of <O, dO> (scores recomputed from the saved LSE).  With K/V
     of fewer heads, dK/dV are summed over each group of query heads."""
     B, H, N, d, Hkv = _check_kv_heads(q, k, v)
@@ -145,11 +162,12 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    st = lib.fa_backward_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                             do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                             dv.data_ptr(), workspace.data_ptr(),
-                             workspace.numel() * workspace.element_size(),
-                             B, H, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    keep, sl = _seqlens_ptr(seqlens, B, q.device)
+    st = lib.fa_backward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                dv.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), sl,
+                                B, H, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_backward")
     return dq, dk, dv

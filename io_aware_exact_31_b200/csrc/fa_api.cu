@@ -86,8 +86,8 @@ fa_status check_heads(int H, int Hkv) {
 
 template <int D>
 fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const void* V, void* O,
-                         float* LSE, int B, int H, int Hkv, int N, float scale, int causal,
-                         cudaStream_t stream) {
+                         float* LSE, int B, int H, int Hkv, int N, const int* seqlens,
+                         float scale, int causal, cudaStream_t stream) {
     using C = FwdCfg<D>;
     CUtensorMap mq, mk, mv;
     const uint64_t depth = static_cast<uint64_t>(B) * H;
@@ -114,6 +114,7 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     p.n_heads = B * H;
     p.H = H;
     p.group = H / Hkv;
+    p.seqlens = seqlens;
     p.n_pairs = (N + 2 * FWD_BM - 1) / (2 * FWD_BM);
     const long long n_ctas = static_cast<long long>(p.n_pairs) * p.n_heads;
     if (n_ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
@@ -154,10 +155,11 @@ using namespace fa;
 
 extern "C" {
 
-fa_status fa_forward_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                         int H, int H_kv, int N, int d, float scale, int causal,
-                         cudaStream_t stream) {
+fa_status fa_forward_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                            const int* seqlens, int B, int H, int H_kv, int N, int d,
+                            float scale, int causal, cudaStream_t stream) {
     if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
         return FA_ERR_INVALID_ARG;
     fa_status st = check_shape(B, H, N, d, scale);
@@ -165,9 +167,16 @@ fa_status fa_forward_gqa(const void* Q, const void* K, const void* V, void* O, f
     if ((st = check_heads(H, H_kv)) != FA_OK) return st;
     DeviceState* ds = current_device(&st);
     if (!ds) return st;
-    return d == 128
-               ? launch_forward<128>(ds, Q, K, V, O, LSE, B, H, H_kv, N, scale, causal, stream)
-               : launch_forward<64>(ds, Q, K, V, O, LSE, B, H, H_kv, N, scale, causal, stream);
+    return d == 128 ? launch_forward<128>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens, scale,
+                                          causal, stream)
+                    : launch_forward<64>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens, scale,
+                                         causal, stream);
+}
+
+fa_status fa_forward_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                         int H, int H_kv, int N, int d, float scale, int causal,
+                         cudaStream_t stream) {
+    return fa_forward_varlen(Q, K, V, O, LSE, nullptr, B, H, H_kv, N, d, scale, causal, stream);
 }
 
 fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
@@ -180,12 +189,14 @@ size_t fa_backward_workspace_bytes(int B, int H, int N, int d) {
     return bwd_workspace_bytes(B, H, N, d);
 }
 
-fa_status fa_backward_gqa(const void* Q, const void* K, const void* V, const void* O,
-                          const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
-                          void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int N,
-                          int d, float scale, int causal, cudaStream_t stream) {
+fa_status fa_backward_varlen(const void* Q, const void* K, const void* V, const void* O,
+                             const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                             void* workspace, size_t workspace_bytes, const int* seqlens, int B,
+                             int H, int H_kv, int N, int d, float scale, int causal,
+                             cudaStream_t stream) {
     if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace)
         return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
     const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
     for (const void* p : ptrs)
         if (!aligned16(p)) return FA_ERR_INVALID_ARG;
@@ -200,10 +211,18 @@ fa_status fa_backward_gqa(const void* Q, const void* K, const void* V, const voi
         if (!bwd_set_attributes(d)) return FA_ERR_CUDA;
         ds->bwd_attr[di] = true;
     }
-    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, H_kv, N, d, scale, causal,
-                      ds->err, stream)
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, H_kv, N, d, seqlens,
+                      scale, causal, ds->err, stream)
                ? FA_OK
                : FA_ERR_CUDA;
+}
+
+fa_status fa_backward_gqa(const void* Q, const void* K, const void* V, const void* O,
+                          const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                          void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int N,
+                          int d, float scale, int causal, cudaStream_t stream) {
+    return fa_backward_varlen(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes,
+                              nullptr, B, H, H_kv, N, d, scale, causal, stream);
 }
 
 fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -320,8 +339,8 @@ extern "C" fa_status fa_backward_noalloc(const void* Q, const void* K, const voi
     // Same three kernels as fa_backward; the preprocess kernel rewrites every
     // byte of the scratch the later kernels read (D, LSE and the zeroed fp32
     // dQ accumulator), so what an earlier call left there does not matter.
-    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, scratch, B, H, H, N, d, scale, causal,
-                      ds->err, stream)
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, scratch, B, H, H, N, d, nullptr, scale,
+                      causal, ds->err, stream)
                ? FA_OK
                : FA_ERR_CUDA;
 }

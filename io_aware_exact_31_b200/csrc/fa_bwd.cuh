@@ -91,6 +91,7 @@ struct BwdParams {
     __nv_bfloat16* dV;
     int N, Npad, n_q_blocks;
     int H, group;        // query heads per batch; query heads per K/V head
+    const int* seqlens;  // [B] real tokens per batch (device), or null
     float scale, scale_log2;
     int causal;
     uint32_t* err;
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(256)
 fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                   const float* __restrict__ LSE, float* __restrict__ Dvec,
                   float* __restrict__ LSE2, float* __restrict__ dQacc, int N, int Npad,
-                  long long rows_pad) {
+                  long long rows_pad, const int* __restrict__ seqlens, int H) {
     constexpr int TPR = D / 8;  // threads per row, 8 bf16 (16 B) each
     const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int sub = threadIdx.x % TPR;
@@ -112,8 +113,9 @@ fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __re
     for (long long r = tid / TPR; r < rows_pad; r += stride) {
         const long long bh = r / Npad;
         const int i = static_cast<int>(r % Npad);
+        const int len = seqlens ? min(max(seqlens[bh / H], 0), N) : N;
         float acc = 0.f;
-        if (i < N) {
+        if (i < len) {
             const size_t off = (static_cast<size_t>(bh) * N + i) * D + sub * 8;
             const uint4 a = *reinterpret_cast<const uint4*>(O + off);
             const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
@@ -131,7 +133,7 @@ fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __re
         for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o, TPR);
         if (sub == 0) {
             Dvec[r] = acc;
-            LSE2[r] = (i < N) ? LSE[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : 0.f;
+            LSE2[r] = (i < len) ? LSE[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : 0.f;
         }
         float4* z = reinterpret_cast<float4*>(dQacc + static_cast<size_t>(r) * D);
 #pragma unroll
@@ -198,8 +200,12 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     const int bq0 = blockIdx.z * p.H + blockIdx.y * p.group;  // first query head of the group
     const int kb = blockIdx.x;  // key block; causal: block 0 has the most work and starts first
     const int k0 = kb * BWD_BN;
+    // Padded batches: only the first len tokens are real; a key block past len
+    // has zero gradients, query blocks past len contribute nothing.
+    const int len = p.seqlens ? min(max(__ldg(p.seqlens + blockIdx.z), 0), p.N) : p.N;
+    const bool padding_cta = k0 >= len;
     const int i_begin = p.causal ? kb : 0;  // first query block that sees this key block
-    const int nq = p.n_q_blocks - i_begin;  // query blocks per query head
+    const int nq = padding_cta ? 0 : (len + BWD_BM - 1) / BWD_BM - i_begin;  // per query head
     const int n_iter = nq * p.group;
     // iteration it -> (query head, query block)
     auto q_head = [&](int it) { return bq0 + it / nq; };
@@ -239,7 +245,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     } else if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
         regs_decrease<BWD_REGS_CONTROL>();
-        if (lane == 0) {
+        if (lane == 0 && !padding_cta) {
             tma_prefetch_desc(&mapQ);
             tma_prefetch_desc(&mapK);
             tma_prefetch_desc(&mapV);
@@ -276,7 +282,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         regs_decrease<BWD_REGS_CONTROL>();
-        if (lane == 0) {
+        if (lane == 0 && !padding_cta) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);  // S^T, dP^T
             const uint32_t id_kn = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
             const uint32_t id_q = idesc_bf16(128, D, true, true);      // dQ (A, B MN-major)
@@ -408,7 +414,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             }
             const uint32_t vL = smem_u32(smem + C::OFF_VEC + s * 1024) + 256 * half;
             const bool need_mask =
-                (key >= p.N) || (q0 + BWD_BM > p.N) || (p.causal && qh < k0 + BWD_BN);
+                (key >= len) || (q0 + BWD_BM > len) || (p.causal && qh < k0 + BWD_BN);
 #pragma unroll
             for (int c4 = 0; c4 < 16; ++c4) {
                 const float4 l4 = ld_shared_v4f(vL + 16 * c4);
@@ -424,7 +430,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const int q = qh + c;
-                    if (key >= p.N || q >= p.N || q < qlim) pv[c] = 0.f;
+                    if (key >= len || q >= len || q < qlim) pv[c] = 0.f;
                 }
             }
             if (C::P_ALIAS) {
@@ -516,7 +522,17 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         if (ok && n_iter > 0) ok = phase_dQr(n_iter - 1);
 
         // ---- dK, dV epilogue (lane = key)
-        if (ok && mbar_wait_warp(&bars->dkdv_full, 0, g, 36)) {
+        if (padding_cta) {
+            constexpr int HC = D / 2;
+            if (key < p.N) {
+                const size_t off = (static_cast<size_t>(bkv) * p.N + key) * D + HC * half;
+#pragma unroll
+                for (int c = 0; c < HC; c += 8) {
+                    st_global_v4(p.dV + off + c, 0u, 0u, 0u, 0u);
+                    st_global_v4(p.dK + off + c, 0u, 0u, 0u, 0u);
+                }
+            }
+        } else if (ok && mbar_wait_warp(&bars->dkdv_full, 0, g, 36)) {
             tc_fence_after();
             constexpr int HC = D / 2;
             const bool valid = key < p.N;
@@ -572,7 +588,8 @@ inline bool bwd_set_attributes(int d) {
 template <int D>
 bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                   const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
-                  int Hkv, int N, float scale, int causal, uint32_t* err, cudaStream_t stream) {
+                  int Hkv, int N, const int* seqlens, float scale, int causal, uint32_t* err,
+                  cudaStream_t stream) {
     const int Npad = static_cast<int>(round_up_128(N));
     const long long rows_pad = static_cast<long long>(B) * H * Npad;
     float* Dvec = static_cast<float*>(workspace);
@@ -583,7 +600,7 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         const int blocks = static_cast<int>(std::min<long long>((threads + 255) / 256, 148LL * 16));
         fa_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, Dvec,
-            LSE2, dQacc, N, Npad, rows_pad);
+            LSE2, dQacc, N, Npad, rows_pad, seqlens, H);
         if (cudaGetLastError() != cudaSuccess) return false;
     }
     {
@@ -605,6 +622,7 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         p.n_q_blocks = Npad / 128;
         p.H = H;
         p.group = H / Hkv;
+        p.seqlens = seqlens;
         p.scale = scale;
         p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
         p.causal = causal ? 1 : 0;
@@ -626,12 +644,12 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
 
 inline bool bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                        const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
-                       int Hkv, int N, int d, float scale, int causal, uint32_t* err,
-                       cudaStream_t stream) {
+                       int Hkv, int N, int d, const int* seqlens, float scale, int causal,
+                       uint32_t* err, cudaStream_t stream) {
     return d == 128 ? bwd_launch_t<128>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N,
-                                        scale, causal, err, stream)
+                                        seqlens, scale, causal, err, stream)
                     : bwd_launch_t<64>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N,
-                                       scale, causal, err, stream);
+                                       seqlens, scale, causal, err, stream);
 }
 
 }  // namespace fa

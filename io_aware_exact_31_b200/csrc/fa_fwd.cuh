@@ -72,6 +72,7 @@ struct FwdParams {
     int n_heads;        // B * H (query heads)
     int H;              // query heads per batch
     int group;          // query heads per K/V head (H / H_kv; 1 = plain multi-head)
+    const int* seqlens; // [B] real tokens per batch (device), or null: all N are real
     int n_pairs;        // ceil(N / 256)
     uint32_t* err;      // device error word
 };
@@ -114,12 +115,17 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     // K/V head of this query head (grouped-query attention; = bh when group = 1).
     const int bkv = (bh / p.H) * (p.H / p.group) + (bh % p.H) / p.group;
     const int q0 = pair * 2 * FWD_BM;
+    // Padded batches: tokens >= len of this batch are padding -- masked as
+    // keys, zero output as queries; key blocks past len are never loaded.
+    const int len = p.seqlens ? min(max(__ldg(p.seqlens + bh / p.H), 0), p.N) : p.N;
+    const int n_kv = (len + FWD_BN - 1) / FWD_BN;
+    const bool padding_cta = q0 >= len;  // all rows of this CTA are padding
     // Key blocks each tile needs: causal tiles stop at their diagonal block.
     int n_tile[2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int last_row = q0 + (t + 1) * FWD_BM - 1;
-        n_tile[t] = p.causal ? min(last_row / FWD_BN + 1, p.n_kv_blocks) : p.n_kv_blocks;
+        n_tile[t] = padding_cta ? 0 : p.causal ? min(last_row / FWD_BN + 1, n_kv) : n_kv;
     }
     const int n_blocks = n_tile[1];  // n_tile[0] <= n_tile[1] <= n_tile[0] + 1
 
@@ -157,7 +163,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     } else if (warp == 9) {
         regs_decrease<FWD_REGS_CONTROL>();
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (lane == 0 && !padding_cta) {
             tma_prefetch_desc(&mapQ);
             tma_prefetch_desc(&mapK);
             tma_prefetch_desc(&mapV);
@@ -207,7 +213,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         regs_decrease<FWD_REGS_CONTROL>();
-        if (lane == 0) {
+        if (lane == 0 && !padding_cta) {
             const uint32_t idS = idesc_bf16(128, FWD_BN, false, false);  // S = Q K^T
             const uint32_t idO = idesc_bf16(128, D, false, true);        // O += P V (V MN-major)
             const uint32_t sQ = smem_u32(smem + C::OFF_Q);
@@ -313,10 +319,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
             const int key0 = j * FWD_BN;
             // Mask keys past the end and (causal) keys after the query.
-            const bool tail = key0 + FWD_BN > p.N;
+            const bool tail = key0 + FWD_BN > len;
             const bool diag = p.causal && key0 + FWD_BN - 1 > tile_first_q;
             if (tail || diag) {
-                const int lim = p.causal ? min(q + 1, p.N) : p.N;  // valid keys: key < lim
+                const int lim = p.causal ? min(q + 1, len) : len;  // valid keys: key < lim
 #pragma unroll
                 for (int i = 0; i < 128; ++i)
                     if (key0 + i >= lim) s[i] = -INFINITY;
@@ -398,9 +404,18 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             }
         }
         // ------------------------------------------------------------ epilogue
-        if (ok && mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t)) {
+        if (padding_cta) {
+            // Padding query rows: O = 0, LSE = 0.
+            if (q < p.N) {
+                __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + q) * D;
+#pragma unroll
+                for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
+                p.LSE[static_cast<size_t>(bh) * p.N + q] = 0.f;
+            }
+        } else if (ok && mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t)) {
             tc_fence_after();
-            const float inv_l = 1.f / lr;
+            const bool real = q < len;  // padding rows of a partly padded tile get zeros
+            const float inv_l = real ? 1.f / lr : 0.f;
             const bool valid = q < p.N;
             __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + (valid ? q : 0)) * D;
 #pragma unroll 1
@@ -423,7 +438,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             }
             if (valid) {
                 // LSE in natural-log units: (m + log2 l) * ln 2.
-                p.LSE[static_cast<size_t>(bh) * p.N + q] = (m_used + __log2f(l)) * 0.69314718055994531f;
+                p.LSE[static_cast<size_t>(bh) * p.N + q] =
+                    real ? (m_used + __log2f(l)) * 0.69314718055994531f : 0.f;
             }
         }
     }

@@ -55,6 +55,10 @@ def load(path: str | None = None):
                                                  vp, vp]
     lib.oracle_attention_backward_gqa.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64, i64, dbl,
                                                   ip, vp, vp, vp]
+    lib.oracle_attention_forward_varlen.argtypes = [vp, vp, vp, ip, vp, i64, i64, i64, i64, i64,
+                                                    dbl, ip, vp, vp]
+    lib.oracle_attention_backward_varlen.argtypes = [vp, vp, vp, vp, ip, vp, i64, i64, i64, i64,
+                                                     i64, dbl, ip, vp, vp, vp]
     lib.oracle_softmax_partial.argtypes = [vp, i64, vp, i64, vp, vp, vp]
     lib.oracle_softmax_merge.argtypes = [dbl, dbl, vp, dbl, dbl, vp, i64, vp, vp, vp]
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -62,7 +66,8 @@ def load(path: str | None = None):
     for name in ("oracle_attention_forward", "oracle_attention_forward_rows",
                  "oracle_attention_backward", "oracle_softmax_partial",
                  "oracle_softmax_merge", "oracle_attention_forward_gqa",
-                 "oracle_attention_backward_gqa"):
+                 "oracle_attention_backward_gqa", "oracle_attention_forward_varlen",
+                 "oracle_attention_backward_varlen"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -165,6 +170,43 @@ def attention_backward_gqa(Q, K, V, dO, scale: float, causal: bool, lib=None):
                                              N, d, float(scale), int(bool(causal)),
                                              _ptr(dQ), _ptr(dK), _ptr(dV)),
            "oracle_attention_backward_gqa")
+    return dQ, dK, dV
+
+
+def attention_forward_varlen(Q, K, V, seqlens, scale: float, causal: bool, lib=None):
+    """Padded batches: seqlens[b] real tokens per batch (keys beyond masked,
+    padding query rows O = 0, LSE = 0).  K/V may have fewer heads (grouped)."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv) = _as_input(Q), _as_input(K), _as_input(V)
+    assert dt == dk == dv and K.shape == V.shape and Q.ndim == 4
+    B, H, N, d = Q.shape
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    assert sl.shape == (B,)
+    O = np.empty((B, H, N, d), np.float64)
+    LSE = np.empty((B, H, N), np.float64)
+    _check(lib.oracle_attention_forward_varlen(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(sl), B, H,
+                                               K.shape[1], N, d, float(scale), int(bool(causal)),
+                                               _ptr(O), _ptr(LSE)),
+           "oracle_attention_forward_varlen")
+    return O, LSE
+
+
+def attention_backward_varlen(Q, K, V, dO, seqlens, scale: float, causal: bool, lib=None):
+    """Gradients for padded batches (all gradients of padding tokens are 0)."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv), (dO, dd) = (_as_input(Q), _as_input(K), _as_input(V),
+                                           _as_input(dO))
+    assert dt == dk == dv == dd and K.shape == V.shape and Q.shape == dO.shape
+    B, H, N, d = Q.shape
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    assert sl.shape == (B,)
+    dQ = np.empty((B, H, N, d), np.float64)
+    dK = np.empty(K.shape, np.float64)
+    dV = np.empty(K.shape, np.float64)
+    _check(lib.oracle_attention_backward_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), dt, _ptr(sl),
+                                                B, H, K.shape[1], N, d, float(scale),
+                                                int(bool(causal)), _ptr(dQ), _ptr(dK), _ptr(dV)),
+           "oracle_attention_backward_varlen")
     return dQ, dK, dV
 
 

@@ -41,6 +41,12 @@
  *           value heads (H_kv divides H); query head h of a batch attends
  *           with key/value head h / (H / H_kv).  The *_gqa functions take
  *           K, V as [B, H_kv, N, d]; with H_kv = H they are [STD] per head.
+ *   [PAD]   downcodes.com "triton transformer", BERT example: a padding
+ *           mask over the tokens of each sequence.  Reading: seqlens[b] (0 ..
+ *           N) tokens of batch b are real, the rest padding.  Padding keys are
+ *           masked for every query; a padding query row has O = 0, LSE = 0
+ *           and contributes nothing to any gradient.  Equivalently: batch b is
+ *           [STD] on its first seqlens[b] tokens.  seqlens = NULL: all N.
  *
  * Every function returns 0 on success, -1 on a bad argument, -2 if memory
  * could not be allocated.
@@ -73,6 +79,22 @@ static int bad_shape(int64_t B, int64_t H, int64_t N, int64_t d, int dtype)
            (dtype != ORACLE_F64 && dtype != ORACLE_BF16);
 }
 
+/* [PAD]: real tokens of batch b. */
+static int64_t seq_len(const int32_t *seqlens, int64_t b, int64_t N)
+{
+    return seqlens ? seqlens[b] : N;
+}
+
+static int bad_seqlens(const int32_t *seqlens, int64_t B, int64_t N)
+{
+    if (!seqlens)
+        return 0;
+    for (int64_t b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > N)
+            return 1;
+    return 0;
+}
+
 /* [GQA]: key/value head of query head bh = b * H + h. */
 static int64_t kv_head(int64_t bh, int64_t H, int64_t Hkv)
 {
@@ -80,8 +102,8 @@ static int64_t kv_head(int64_t bh, int64_t H, int64_t Hkv)
 }
 
 /*
- * One output row of [STD] for query i (queries of this head start at element
- * q_base, its keys and values at kv_base):
+ * One output row of [STD] for query i over keys j < n_keys (queries of this
+ * head start at element q_base, its keys and values at kv_base):
  *   s_j   = scale * <q_i, k_j>           (s_j = -inf if causal and j > i)
  *   m     = max_j s_j                    ([SAFE])
  *   LSE_i = m + ln sum_j exp(s_j - m)
@@ -90,10 +112,11 @@ static int64_t kv_head(int64_t bh, int64_t H, int64_t Hkv)
  * s is caller-provided scratch of N doubles.
  */
 static void attention_row(const void *Q, const void *K, const void *V, int dtype,
-                          int64_t N, int64_t d, int64_t q_base, int64_t kv_base, int64_t i,
+                          int64_t n_keys, int64_t d, int64_t q_base, int64_t kv_base, int64_t i,
                           double scale, int causal, double *s,
                           double *o_row, double *lse)
 {
+    const int64_t N = n_keys;
     for (int64_t j = 0; j < N; ++j) {
         if (causal && j > i) {
             s[j] = -INFINITY;
@@ -124,14 +147,15 @@ static void attention_row(const void *Q, const void *K, const void *V, int dtype
     }
 }
 
-/* Full forward with [GQA] heads: O [B,H,N,d] and LSE [B,H,N], both double;
- * K, V are [B,Hkv,N,d]. */
-int oracle_attention_forward_gqa(const void *Q, const void *K, const void *V, int dtype,
-                                 int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
-                                 double scale, int causal, double *O, double *LSE)
+/* Full forward with [GQA] heads and [PAD] lengths: O [B,H,N,d] and LSE
+ * [B,H,N], both double; K, V are [B,Hkv,N,d]; seqlens [B] or NULL. */
+int oracle_attention_forward_varlen(const void *Q, const void *K, const void *V, int dtype,
+                                    const int32_t *seqlens, int64_t B, int64_t H, int64_t Hkv,
+                                    int64_t N, int64_t d, double scale, int causal,
+                                    double *O, double *LSE)
 {
     if (!Q || !K || !V || !O || !LSE || bad_shape(B, H, N, d, dtype) ||
-        Hkv < 1 || Hkv > H || H % Hkv != 0)
+        Hkv < 1 || Hkv > H || H % Hkv != 0 || bad_seqlens(seqlens, B, N))
         return -1;
     const int64_t rows = B * H * N;
     int failed = 0;
@@ -147,12 +171,28 @@ int oracle_attention_forward_gqa(const void *Q, const void *K, const void *V, in
             if (!s)
                 continue;
             const int64_t bh = r / N, i = r % N;
-            attention_row(Q, K, V, dtype, N, d, bh * N * d, kv_head(bh, H, Hkv) * N * d, i,
+            const int64_t len = seq_len(seqlens, bh / H, N);
+            if (i >= len) { /* padding query row */
+                for (int64_t c = 0; c < d; ++c)
+                    O[r * d + c] = 0.0;
+                LSE[r] = 0.0;
+                continue;
+            }
+            attention_row(Q, K, V, dtype, len, d, bh * N * d, kv_head(bh, H, Hkv) * N * d, i,
                           scale, causal, s, O + r * d, LSE + r);
         }
         free(s);
     }
     return failed ? -2 : 0;
+}
+
+/* Full forward with [GQA] heads, no padding. */
+int oracle_attention_forward_gqa(const void *Q, const void *K, const void *V, int dtype,
+                                 int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                 double scale, int causal, double *O, double *LSE)
+{
+    return oracle_attention_forward_varlen(Q, K, V, dtype, NULL, B, H, Hkv, N, d, scale, causal,
+                                           O, LSE);
 }
 
 /* Full forward, one key/value head per query head. */
@@ -215,16 +255,19 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
  *   dQ_i  = scale sum_j dS_ij k_j
  *   dK_j  = scale sum_i dS_ij q_i
  * With [GQA] heads the key/value gradients of a key/value head are the sums
- * of these over the query heads that share it.  dQ is double [B,H,N,d];
- * dK, dV are double [B,Hkv,N,d].
+ * of these over the query heads that share it.  With [PAD] lengths each
+ * (batch, head) is the same on its first len tokens (P = 0 outside) and all
+ * gradients of padding tokens are 0.  dQ is double [B,H,N,d]; dK, dV are
+ * double [B,Hkv,N,d].
  */
-int oracle_attention_backward_gqa(const void *Q, const void *K, const void *V, const void *dO,
-                                  int dtype, int64_t B, int64_t H, int64_t Hkv, int64_t N,
-                                  int64_t d, double scale, int causal,
-                                  double *dQ, double *dK, double *dV)
+int oracle_attention_backward_varlen(const void *Q, const void *K, const void *V,
+                                     const void *dO, int dtype, const int32_t *seqlens,
+                                     int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                     double scale, int causal,
+                                     double *dQ, double *dK, double *dV)
 {
     if (!Q || !K || !V || !dO || !dQ || !dK || !dV || bad_shape(B, H, N, d, dtype) ||
-        Hkv < 1 || Hkv > H || H % Hkv != 0)
+        Hkv < 1 || Hkv > H || H % Hkv != 0 || bad_seqlens(seqlens, B, N))
         return -1;
     double *P = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
     double *dS = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
@@ -237,9 +280,13 @@ int oracle_attention_backward_gqa(const void *Q, const void *K, const void *V, c
         dK[e] = 0.0;
         dV[e] = 0.0;
     }
+    for (int64_t e = 0; e < B * H * N * d; ++e)
+        dQ[e] = 0.0;
     for (int64_t bh = 0; bh < B * H; ++bh) {
         const int64_t base = bh * N * d;                        /* Q, dO, dQ */
         const int64_t kv_base = kv_head(bh, H, Hkv) * N * d;    /* K, V, dK, dV */
+        const int64_t N_full = N;
+        const int64_t N = seq_len(seqlens, bh / H, N_full);     /* real tokens */
         /* P row by row, exactly as the forward defines it. */
 #pragma omp parallel for schedule(dynamic, 8)
         for (int64_t i = 0; i < N; ++i) {
@@ -308,6 +355,16 @@ int oracle_attention_backward_gqa(const void *Q, const void *K, const void *V, c
     free(P);
     free(dS);
     return 0;
+}
+
+/* Backward with [GQA] heads, no padding. */
+int oracle_attention_backward_gqa(const void *Q, const void *K, const void *V, const void *dO,
+                                  int dtype, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                                  int64_t d, double scale, int causal,
+                                  double *dQ, double *dK, double *dV)
+{
+    return oracle_attention_backward_varlen(Q, K, V, dO, dtype, NULL, B, H, Hkv, N, d, scale,
+                                            causal, dQ, dK, dV);
 }
 
 /* Backward with one key/value head per query head. */

@@ -406,6 +406,65 @@ def pin_gqa_backward_vs_autograd(lib):
         _close(dV, tv.grad.numpy())
 
 
+# ----------------------------------------------------------------------------
+# Padding pins (downcodes.com "triton transformer", BERT example: padding mask)
+# ----------------------------------------------------------------------------
+
+def _key_mask(seqlens, N, causal):
+    """[B, 1, N, N] boolean: query i may attend key j."""
+    B = len(seqlens)
+    j = torch.arange(N)
+    m = (j[None, :] < torch.tensor(seqlens)[:, None])[:, None, None, :].expand(B, 1, N, N)
+    if causal:
+        m = m & torch.ones(N, N, dtype=torch.bool).tril()
+    return m
+
+
+def pin_padding_forward_vs_torch(lib):
+    """Real rows: torch SDPA (fp64) with a boolean key-padding mask; padding
+    rows: O = 0, LSE = 0."""
+    r = _rng(23)
+    for (B, H, Hkv, N, d, causal, sl) in [(3, 2, 2, 9, 4, False, [9, 5, 1]),
+                                          (2, 4, 2, 12, 8, True, [7, 12])]:
+        Q = r.standard_normal((B, H, N, d))
+        K, V = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+        O, LSE = oracle.attention_forward_varlen(Q, K, V, sl, 0.6, causal, lib=lib)
+        G = H // Hkv
+        tq = torch.from_numpy(Q)
+        tk = torch.from_numpy(np.repeat(K, G, axis=1))
+        tv = torch.from_numpy(np.repeat(V, G, axis=1))
+        mask = _key_mask(sl, N, causal)
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                               scale=0.6)
+        s = (0.6 * tq @ tk.transpose(-1, -2)).masked_fill(~mask, float("-inf"))
+        for b, n in enumerate(sl):
+            _close(O[b, :, :n], ref[b, :, :n].numpy())
+            _close(LSE[b, :, :n], torch.logsumexp(s[b, :, :n], dim=-1).numpy())
+            assert np.all(O[b, :, n:] == 0.0) and np.all(LSE[b, :, n:] == 0.0)
+
+
+def pin_padding_backward_vs_autograd(lib):
+    """torch.autograd (fp64) on real rows only: padding queries contribute
+    nothing, padding tokens get zero gradients."""
+    r = _rng(24)
+    for (B, H, Hkv, N, d, causal, sl) in [(2, 2, 1, 10, 4, True, [6, 10]),
+                                          (2, 2, 2, 8, 4, False, [3, 8])]:
+        Q, dO = (r.standard_normal((B, H, N, d)) for _ in range(2))
+        K, V = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+        tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+        G = H // Hkv
+        mask = _key_mask(sl, N, causal)
+        s = (0.5 * tq @ tk.repeat_interleave(G, dim=1).transpose(-1, -2)).masked_fill(
+            ~mask, float("-inf"))
+        out = torch.softmax(s, dim=-1) @ tv.repeat_interleave(G, dim=1)
+        real = (torch.arange(N)[None, :] < torch.tensor(sl)[:, None])[:, None, :, None]
+        (out * torch.from_numpy(dO) * real).sum().backward()
+        dQ, dK, dV = oracle.attention_backward_varlen(Q, K, V, dO, sl, 0.5, causal, lib=lib)
+        _close(dQ, (tq.grad * real).numpy())
+        _close(dK, tk.grad.numpy())
+        _close(dV, tv.grad.numpy())
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -461,6 +520,12 @@ MUTANTS = {
                               "return (bh / H) * Hkv + (bh % H) % Hkv;", 0),
     "gqa_dK_overwrites": ("dK[kv_base + j * d + c] += scale * acc_k;",
                           "dK[kv_base + j * d + c] = scale * acc_k;", 0),
+    "pad_keys_not_masked": ("attention_row(Q, K, V, dtype, len, d,",
+                            "attention_row(Q, K, V, dtype, N, d,", 0),
+    "pad_query_off_by_one": ("if (i >= len) { /* padding query row */",
+                             "if (i > len) { /* padding query row */", 0),
+    "pad_bwd_uses_full_length": ("const int64_t N = seq_len(seqlens, bh / H, N_full);",
+                                 "const int64_t N = N_full;", 0),
     "exp_sign": ("s[j] = exp(s[j] - m); /* exp(-inf)", "s[j] = exp(m - s[j]); /* exp(-inf)", 0),
     "bwd_drop_scale_in_scores": ("s[j] = scale * acc;", "s[j] = acc;", 1),
     "bwd_drop_D": ("ds[j] = P[i * N + j] * (ds[j] - D);", "ds[j] = P[i * N + j] * ds[j];", 0),
