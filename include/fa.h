@@ -89,6 +89,23 @@ fa_status fa_forward_varlen(const void *Q, const void *K, const void *V, void *O
                             float scale, int causal, cudaStream_t stream);
 
 /*
+ * FP8 forward (the FlashAttention-3 direction of the pages: FP8 compute,
+ * systems-analysis.info "FlashAttention-2 (VI)", FlashAttention-3 section).
+ *   Q8, K8, V8 : [B,H,N,d] / [B,H_kv,N,d] E4M3 bytes (__nv_fp8_e4m3); the
+ *                real inputs are Q8 * descale_q, K8 * descale_k, V8 * descale_v
+ *                (per-tensor dequantisation scales, finite and > 0)
+ *   O, LSE     : as fa_forward (bf16 O, fp32 natural-log LSE of the scaled
+ *                real scores)
+ * The S = Q K^T and P.V products run on the tensor core in E4M3 with fp32
+ * accumulation; P is rounded to E4M3 (3 mantissa bits) for the P.V product and
+ * O is normalised by the sum of the same rounded weights.  d must be 128
+ * (FA_ERR_UNSUPPORTED otherwise).  No backward.
+ */
+fa_status fa_forward_fp8(const void *Q8, const void *K8, const void *V8, void *O, float *LSE,
+                         float descale_q, float descale_k, float descale_v, int B, int H,
+                         int H_kv, int N, int d, float scale, int causal, cudaStream_t stream);
+
+/*
  * Device workspace fa_backward needs, in bytes (0 on invalid shapes).  It holds
  * D_i = <dO_i, O_i>, LSE in base-2 units and the fp32 dQ accumulator, each
  * padded to a multiple of 128 rows per head.

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 
 # Every entry point include/fa.h declares.
-EXPORTS = ("fa_forward", "fa_forward_gqa", "fa_forward_varlen", "fa_backward_workspace_bytes",
+EXPORTS = ("fa_forward", "fa_forward_gqa", "fa_forward_varlen", "fa_forward_fp8",
+           "fa_backward_workspace_bytes",
            "fa_backward", "fa_backward_gqa", "fa_backward_varlen", "fa_backward_noalloc",
            "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_str", "fa_version")
 
@@ -61,6 +62,8 @@ def load_library(path: str | None = None):
     lib.fa_backward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, i, i, i, i,
                                        i, f, i, vp]
     lib.fa_backward_varlen.restype = i
+    lib.fa_forward_fp8.argtypes = [vp, vp, vp, vp, vp, f, f, f, i, i, i, i, i, f, i, vp]
+    lib.fa_forward_fp8.restype = i
     lib.fa_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_backward_noalloc.restype = i
     lib.fa_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -144,6 +147,30 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fa
                                           int(bool(causal)), _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_forward")
+    return o, l
+
+
+def forward_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
+                causal: bool = False, scale: float | None = None, out=None, lse=None,
+                stream=None):
+    """FP8 forward: q8/k8/v8 are torch.float8_e4m3fn [B,H,N,128] ([B,H_kv,N,128]
+    for K/V); the real inputs are q8 * descale_q etc.  Returns bf16 O and LSE."""
+    for t in (q8, k8, v8):
+        if not t.is_cuda or t.dtype != torch.float8_e4m3fn or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("inputs must be contiguous float8_e4m3fn CUDA tensors [B, H, N, d]")
+    B, H, N, d = q8.shape
+    Hkv = k8.shape[1]
+    if k8.shape != v8.shape or k8.shape[0] != B or k8.shape[2:] != q8.shape[2:]:
+        raise ValueError("K/V shape incompatible with Q")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty(q8.shape, device=q8.device, dtype=torch.bfloat16) if out is None else out
+    l = torch.empty((B, H, N), device=q8.device, dtype=torch.float32) if lse is None else lse
+    st = load_library().fa_forward_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), o.data_ptr(),
+                                       l.data_ptr(), float(descale_q), float(descale_k),
+                                       float(descale_v), B, H, Hkv, N, d, scale, int(bool(causal)),
+                                       _stream_handle(stream))
+    if st != FA_OK:
+        raise FaError(st, "fa_forward_fp8")
     return o, l
 
 

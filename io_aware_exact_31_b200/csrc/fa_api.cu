@@ -23,7 +23,7 @@ struct DeviceState {
     bool checked = false;
     bool supported = false;
     uint32_t* err = nullptr;  // device address of g_err_word on this device
-    bool fwd_attr[2] = {false, false};
+    bool fwd_attr[3] = {false, false, false};  // d = 64, d = 128, d = 128 E4M3
     bool bwd_attr[2] = {false, false};
 };
 
@@ -84,21 +84,28 @@ fa_status check_heads(int H, int Hkv) {
     return FA_OK;
 }
 
-template <int D>
+// scale_qk multiplies the scores (dequant scales of E4M3 Q and K), scale_v
+// the output (dequant scale of E4M3 V); both 1 for bf16 inputs.
+template <int D, bool F8>
 fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const void* V, void* O,
                          float* LSE, int B, int H, int Hkv, int N, const int* seqlens,
-                         float scale, int causal, cudaStream_t stream) {
-    using C = FwdCfg<D>;
+                         float scale, int causal, cudaStream_t stream, double scale_qk = 1.0,
+                         float scale_v = 1.f) {
+    using C = FwdCfg<D, F8>;
     CUtensorMap mq, mk, mv;
     const uint64_t depth = static_cast<uint64_t>(B) * H;
     const uint64_t depth_kv = static_cast<uint64_t>(B) * Hkv;
-    if (!make_map_bf16_3d(&mq, Q, depth, N, D, FWD_BM) ||
-        !make_map_bf16_3d(&mk, K, depth_kv, N, D, FWD_BN) ||
-        !make_map_bf16_3d(&mv, V, depth_kv, N, D, FWD_BN))
-        return FA_ERR_CUDA;
-    const int di = (D == 128) ? 1 : 0;
+    const bool maps_ok =
+        F8 ? (make_map_u8_3d(&mq, Q, depth, N, D, FWD_BM) &&
+              make_map_u8_3d(&mk, K, depth_kv, N, D, FWD_BN) &&
+              make_map_u8_3d(&mv, V, depth_kv, N, D, FWD_BN))
+           : (make_map_bf16_3d(&mq, Q, depth, N, D, FWD_BM) &&
+              make_map_bf16_3d(&mk, K, depth_kv, N, D, FWD_BN) &&
+              make_map_bf16_3d(&mv, V, depth_kv, N, D, FWD_BN));
+    if (!maps_ok) return FA_ERR_CUDA;
+    const int di = F8 ? 2 : (D == 128) ? 1 : 0;
     if (!ds->fwd_attr[di]) {
-        if (cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(fa_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES) != cudaSuccess)
             return FA_ERR_CUDA;
         ds->fwd_attr[di] = true;
@@ -108,7 +115,8 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     p.LSE = LSE;
     p.N = N;
     p.n_kv_blocks = (N + FWD_BN - 1) / FWD_BN;
-    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * scale_qk * 1.4426950408889634);
+    p.o_scale = scale_v;
     p.causal = causal ? 1 : 0;
     p.err = ds->err;
     p.n_heads = B * H;
@@ -119,7 +127,7 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     const long long n_ctas = static_cast<long long>(p.n_pairs) * p.n_heads;
     if (n_ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
     dim3 grid(static_cast<unsigned>(n_ctas));
-    fa_fwd_kernel<D><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+    fa_fwd_kernel<D, F8><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -167,10 +175,29 @@ fa_status fa_forward_varlen(const void* Q, const void* K, const void* V, void* O
     if ((st = check_heads(H, H_kv)) != FA_OK) return st;
     DeviceState* ds = current_device(&st);
     if (!ds) return st;
-    return d == 128 ? launch_forward<128>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens, scale,
-                                          causal, stream)
-                    : launch_forward<64>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens, scale,
-                                         causal, stream);
+    return d == 128 ? launch_forward<128, false>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens,
+                                                 scale, causal, stream)
+                    : launch_forward<64, false>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens,
+                                                scale, causal, stream);
+}
+
+fa_status fa_forward_fp8(const void* Q8, const void* K8, const void* V8, void* O, float* LSE,
+                         float descale_q, float descale_k, float descale_v, int B, int H,
+                         int H_kv, int N, int d, float scale, int causal, cudaStream_t stream) {
+    if (!Q8 || !K8 || !V8 || !O || !LSE) return FA_ERR_INVALID_ARG;
+    if (!aligned16(Q8) || !aligned16(K8) || !aligned16(V8) || !aligned16(O) || !aligned16(LSE))
+        return FA_ERR_INVALID_ARG;
+    fa_status st = check_shape(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if ((st = check_heads(H, H_kv)) != FA_OK) return st;
+    for (float f : {descale_q, descale_k, descale_v})
+        if (!std::isfinite(f) || !(f > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    return launch_forward<128, true>(ds, Q8, K8, V8, O, LSE, B, H, H_kv, N, nullptr, scale,
+                                     causal, stream,
+                                     static_cast<double>(descale_q) * descale_k, descale_v);
 }
 
 fa_status fa_forward_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,

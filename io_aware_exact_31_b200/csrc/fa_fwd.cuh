@@ -46,13 +46,19 @@ constexpr uint32_t FWD_REGS_SOFTMAX = 216;
 constexpr uint32_t FWD_REGS_CONTROL = 72;
 constexpr float FWD_RESCALE_TAU = 8.0f;  // log2 units: keep a stale row max while p <= 2^8
 
-template <int D>
+// F8: Q, K, V and P in E4M3 (kind::f8f6f4 MMAs); otherwise bf16 (kind::f16).
+template <int D, bool F8 = false>
 struct FwdCfg {
-    static constexpr int TILE_BYTES = FWD_BM * D * 2;  // one Q, K or V tile (bf16)
-    static constexpr int NK = 3;                       // K ring depth
-    static constexpr int NV = (D == 128) ? 2 : 3;      // V ring depth
-    static constexpr int PREFETCH = 2;                 // L2 prefetch distance beyond the rings
-    static constexpr int CHUNKS = D / 64;              // 64-wide (128 B) TMA boxes per tile
+    static constexpr int ESZ = F8 ? 1 : 2;                 // operand bytes per element
+    static constexpr int TILE_BYTES = FWD_BM * D * ESZ;    // one Q, K or V tile
+    static constexpr int NK = 3;                           // K ring depth
+    static constexpr int NV = (D * ESZ == 256) ? 2 : 3;    // V ring depth
+    static constexpr int PREFETCH = 2;                     // L2 prefetch distance beyond the rings
+    static constexpr int BOX_ELEMS = 128 / ESZ;            // elements per 128-B TMA box row
+    static constexpr int CHUNKS = D / BOX_ELEMS;           // TMA boxes per tile
+    static constexpr int KSTEP = 32 / ESZ;                 // MMA k per instruction (32 B)
+    static constexpr int PV_PER_HALF = 64 / KSTEP;         // P.V instructions per 64 keys
+    static constexpr int P_COLS_HALF = 64 * ESZ / 4;       // TMEM columns of 64 keys of P
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
@@ -67,7 +73,8 @@ struct FwdParams {
     float* LSE;
     int N;              // sequence length
     int n_kv_blocks;    // ceil(N / 128)
-    float scale_log2;   // scale * log2(e)
+    float scale_log2;   // scale * log2(e) (times the Q and K dequant scales for E4M3)
+    float o_scale;      // V dequant scale for E4M3 inputs (1 for bf16)
     int causal;
     int n_heads;        // B * H (query heads)
     int H;              // query heads per batch
@@ -85,11 +92,11 @@ struct FwdBars {
     uint64_t s_full[2], p_full[2][2], o_full[2];  // p_full[tile][key half]
 };
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
               const __grid_constant__ CUtensorMap mapV, const FwdParams p) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -173,7 +180,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(smem + C::OFF_Q + t * C::TILE_BYTES + c * 16384, &mapQ,
-                                &bars->q_full, c * 64, q0 + t * FWD_BM, bh);
+                                &bars->q_full, c * C::BOX_ELEMS, q0 + t * FWD_BM, bh);
             // K(j) and V(j) go to their own rings; L2 is asked for the tiles
             // PREFETCH blocks beyond what the rings hold.
             int k_issued = 0, v_issued = 0;
@@ -184,14 +191,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(smem + C::OFF_K + sk * C::TILE_BYTES + c * 16384, &mapK,
-                                &bars->k_full[sk], c * 64, j * FWD_BN, bkv);
+                                &bars->k_full[sk], c * C::BOX_ELEMS, j * FWD_BN, bkv);
                 k_issued = j + 1;
                 const int jp = j + C::NK + C::PREFETCH - 1;
                 if (jp < n_blocks) {
 #pragma unroll
                     for (int c = 0; c < C::CHUNKS; ++c) {
-                        tma_prefetch_l2_3d(&mapK, c * 64, jp * FWD_BN, bkv);
-                        tma_prefetch_l2_3d(&mapV, c * 64, jp * FWD_BN, bkv);
+                        tma_prefetch_l2_3d(&mapK, c * C::BOX_ELEMS, jp * FWD_BN, bkv);
+                        tma_prefetch_l2_3d(&mapV, c * C::BOX_ELEMS, jp * FWD_BN, bkv);
                     }
                 }
                 if (j >= C::NV && !mbar_wait(&bars->v_empty[sv], ((j / C::NV) & 1) ^ 1, g, 2)) break;
@@ -199,7 +206,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
 #pragma unroll
                 for (int c = 0; c < C::CHUNKS; ++c)
                     tma_load_3d(smem + C::OFF_V + sv * C::TILE_BYTES + c * 16384, &mapV,
-                                &bars->v_full[sv], c * 64, j * FWD_BN, bkv);
+                                &bars->v_full[sv], c * C::BOX_ELEMS, j * FWD_BN, bkv);
                 v_issued = j + 1;
             }
             // Never leave the CTA with copies still landing in its shared
@@ -214,32 +221,38 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         // ------------------------------------------------------------ MMA issuer
         regs_decrease<FWD_REGS_CONTROL>();
         if (lane == 0 && !padding_cta) {
-            const uint32_t idS = idesc_bf16(128, FWD_BN, false, false);  // S = Q K^T
-            const uint32_t idO = idesc_bf16(128, D, false, true);        // O += P V (V MN-major)
+            // S = Q K^T (K-major A, B); O += P V (V MN-major)
+            const uint32_t idS = F8 ? idesc_e4m3(128, FWD_BN, false) : idesc_bf16(128, FWD_BN, false, false);
+            const uint32_t idO = F8 ? idesc_e4m3(128, D, true) : idesc_bf16(128, D, false, true);
             const uint32_t sQ = smem_u32(smem + C::OFF_Q);
             const uint32_t sK = smem_u32(smem + C::OFF_K);
             const uint32_t sV = smem_u32(smem + C::OFF_V);
             const uint32_t tS[2] = {tmem + C::TMEM_S0, tmem + C::TMEM_S1};
             const uint32_t tO[2] = {tmem + C::TMEM_O0, tmem + C::TMEM_O1};
 
-            // S_t = Q_t K_j^T : K-major A and B, D/16 steps of k = 16.
+            // S_t = Q_t K_j^T : K-major A and B, steps of 32 bytes along d.
             auto issue_S = [&](int t, int s) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < D / C::KSTEP; ++kk) {
                     const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
                     const uint64_t a = sdesc_sw128(sQ + t * C::TILE_BYTES + koff, 16, 1024);
                     const uint64_t b = sdesc_sw128(sK + s * C::TILE_BYTES + koff, 16, 1024);
-                    mma_ss(tS[t], a, b, idS, kk > 0);
+                    if constexpr (F8) mma_ss_f8(tS[t], a, b, idS, kk > 0);
+                    else mma_ss(tS[t], a, b, idS, kk > 0);
                 }
             };
             // O_t (+)= P_t V_j for keys [64h, 64h + 64): P from TMEM (8 columns
-            // per k = 16), V MN-major.  The two halves are issued as soon as the
-            // softmax warps release each half of P.
+            // per instruction), V MN-major (KSTEP key rows of 128 B per step).
+            // The two halves are issued as soon as the softmax warps release
+            // each half of P.
             auto issue_PV_half = [&](int t, int s, int h, bool acc) {
 #pragma unroll
-                for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
-                    const uint64_t b = sdesc_sw128(sV + s * C::TILE_BYTES + kk * 2048, 16384, 1024);
-                    mma_ts(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
+                for (int i = 0; i < C::PV_PER_HALF; ++i) {
+                    const int kk = h * C::PV_PER_HALF + i;
+                    const uint64_t b = sdesc_sw128(sV + s * C::TILE_BYTES + kk * C::KSTEP * 128,
+                                                   16384, 1024);
+                    if constexpr (F8) mma_ts_f8(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
+                    else mma_ts(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
                 }
             };
 
@@ -371,7 +384,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             // weights the tensor core multiplies V with, used to normalise O, so
             // that O = sum p~ v / sum p~ is an exact convex combination of value
             // rows (a row dominated by one key returns that value row exactly).
-            // P goes to TMEM as bf16 pairs (key 2c in the low half of column c).
+            // P goes to TMEM as bf16 pairs (key 2c in the low half of column c),
+            // or for E4M3 operands four per column (key 4c + b in byte b).
             // Packed f32x2 arithmetic, four independent accumulators per sum.
             const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(-m_sub, -m_sub);
             float2 ae[4], ar[4];
@@ -385,11 +399,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     const float2 x =
                         __ffma2_rn(make_float2(s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]), sl2v, negm);
                     const float2 pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                    pk[i] = pack_bf16x2(pe.x, pe.y);
                     ae[i % 4] = __fadd2_rn(ae[i % 4], pe);
-                    ar[i % 4] = __fadd2_rn(ar[i % 4], unpack_bf16x2(pk[i]));
+                    if constexpr (F8) {
+                        // four E4M3 per column: keys 4c..4c+3 in bytes 0..3
+                        const uint32_t h16 = pack_e4m3x2(pe.x, pe.y);
+                        if (i & 1) {
+                            pk[i / 2] |= h16 << 16;
+                            float2 a, b;
+                            unpack_e4m3x4(pk[i / 2], a, b);
+                            ar[i % 4] = __fadd2_rn(ar[i % 4], __fadd2_rn(a, b));
+                        } else {
+                            pk[i / 2] = h16;
+                        }
+                    } else {
+                        pk[i] = pack_bf16x2(pe.x, pe.y);
+                        ar[i % 4] = __fadd2_rn(ar[i % 4], unpack_bf16x2(pk[i]));
+                    }
                 }
-                tmem_st32(tS + h * 32, pk);
+                if constexpr (F8) tmem_st16(tS + h * C::P_COLS_HALF, pk);
+                else tmem_st32(tS + h * C::P_COLS_HALF, pk);
                 // Release this half of P: the tensor core starts on keys
                 // [64h, 64h + 64) while the other half is still being computed.
                 tmem_st_wait();
@@ -415,7 +443,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         } else if (ok && mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t)) {
             tc_fence_after();
             const bool real = q < len;  // padding rows of a partly padded tile get zeros
-            const float inv_l = real ? 1.f / lr : 0.f;
+            const float inv_l = real ? p.o_scale / lr : 0.f;
             const bool valid = q < p.N;
             __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + (valid ? q : 0)) * D;
 #pragma unroll 1

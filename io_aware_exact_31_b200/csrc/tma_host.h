@@ -44,6 +44,22 @@ inline bool make_map_bf16_3d(CUtensorMap* map, const void* base, uint64_t depth,
     return r == CUDA_SUCCESS;
 }
 
+// Same for 8-bit elements (E4M3 stored as bytes): boxes of [1, box_rows, 128].
+inline bool make_map_u8_3d(CUtensorMap* map, const void* base, uint64_t depth, uint64_t rows,
+                           uint64_t cols, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {cols, rows, depth};
+    cuuint64_t strides[2] = {cols, rows * cols};
+    cuuint32_t box[3] = {128, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // A 3-D map over a contiguous [depth, rows, cols] fp32 tensor (cols fastest),
 // boxes of [1, 128, 32] (32 floats = 128 B) with the 128-byte swizzle; used as
 // the destination of shared -> global add-reductions.
