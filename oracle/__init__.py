@@ -59,6 +59,14 @@ def load(path: str | None = None):
                                                     dbl, ip, vp, vp]
     lib.oracle_attention_backward_varlen.argtypes = [vp, vp, vp, vp, ip, vp, i64, i64, i64, i64,
                                                      i64, dbl, ip, vp, vp, vp]
+    u64, u32 = ctypes.c_uint64, ctypes.c_uint32
+    lib.oracle_attention_forward_dropout.argtypes = [vp, vp, vp, ip, vp, i64, i64, i64, i64, i64,
+                                                     dbl, ip, dbl, u64, u32, vp, vp]
+    lib.oracle_attention_backward_dropout.argtypes = [vp, vp, vp, vp, ip, vp, i64, i64, i64, i64,
+                                                      i64, dbl, ip, dbl, u64, u32, vp, vp, vp]
+    lib.oracle_philox4x32_10.argtypes = [vp, vp, vp]
+    lib.oracle_philox4x32_10.restype = None
+    lib.oracle_dropout_keep_mask.argtypes = [i64, i64, i64, dbl, u64, u32, vp]
     lib.oracle_softmax_partial.argtypes = [vp, i64, vp, i64, vp, vp, vp]
     lib.oracle_softmax_merge.argtypes = [dbl, dbl, vp, dbl, dbl, vp, i64, vp, vp, vp]
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -67,7 +75,8 @@ def load(path: str | None = None):
                  "oracle_attention_backward", "oracle_softmax_partial",
                  "oracle_softmax_merge", "oracle_attention_forward_gqa",
                  "oracle_attention_backward_gqa", "oracle_attention_forward_varlen",
-                 "oracle_attention_backward_varlen"):
+                 "oracle_attention_backward_varlen", "oracle_attention_forward_dropout",
+                 "oracle_attention_backward_dropout", "oracle_dropout_keep_mask"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -208,6 +217,75 @@ def attention_backward_varlen(Q, K, V, dO, seqlens, scale: float, causal: bool, 
                                                 int(bool(causal)), _ptr(dQ), _ptr(dK), _ptr(dV)),
            "oracle_attention_backward_varlen")
     return dQ, dK, dV
+
+
+def _seqlens_arg(seqlens, B):
+    if seqlens is None:
+        return None, None
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    assert sl.shape == (B,)
+    return sl, _ptr(sl)
+
+
+def attention_forward_dropout(Q, K, V, scale: float, causal: bool, p_drop: float, seed: int,
+                              offset: int = 0, seqlens=None, lib=None):
+    """Forward with attention dropout (Philox-4x32-10 keep mask; see the C
+    file).  K/V may have fewer heads; seqlens optional.  p_drop = 0 is the
+    plain forward."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv) = _as_input(Q), _as_input(K), _as_input(V)
+    assert dt == dk == dv and K.shape == V.shape and Q.ndim == 4
+    B, H, N, d = Q.shape
+    sl, slp = _seqlens_arg(seqlens, B)
+    O = np.empty((B, H, N, d), np.float64)
+    LSE = np.empty((B, H, N), np.float64)
+    _check(lib.oracle_attention_forward_dropout(_ptr(Q), _ptr(K), _ptr(V), dt, slp, B, H,
+                                                K.shape[1], N, d, float(scale), int(bool(causal)),
+                                                float(p_drop), int(seed), int(offset),
+                                                _ptr(O), _ptr(LSE)),
+           "oracle_attention_forward_dropout")
+    return O, LSE
+
+
+def attention_backward_dropout(Q, K, V, dO, scale: float, causal: bool, p_drop: float, seed: int,
+                               offset: int = 0, seqlens=None, lib=None):
+    """Exact gradient of the dropout forward for the same (p_drop, seed, offset)."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv), (dO, dd) = (_as_input(Q), _as_input(K), _as_input(V),
+                                           _as_input(dO))
+    assert dt == dk == dv == dd and K.shape == V.shape and Q.shape == dO.shape
+    B, H, N, d = Q.shape
+    sl, slp = _seqlens_arg(seqlens, B)
+    dQ = np.empty((B, H, N, d), np.float64)
+    dK = np.empty(K.shape, np.float64)
+    dV = np.empty(K.shape, np.float64)
+    _check(lib.oracle_attention_backward_dropout(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), dt, slp, B,
+                                                 H, K.shape[1], N, d, float(scale),
+                                                 int(bool(causal)), float(p_drop), int(seed),
+                                                 int(offset), _ptr(dQ), _ptr(dK), _ptr(dV)),
+           "oracle_attention_backward_dropout")
+    return dQ, dK, dV
+
+
+def philox4x32_10(counter, key, lib=None):
+    """The four 32-bit output words of Philox-4x32-10 for a 4-word counter and 2-word key."""
+    lib = lib or load()
+    c = np.ascontiguousarray(counter, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    assert c.shape == (4,) and k.shape == (2,)
+    out = np.empty(4, np.uint32)
+    lib.oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def dropout_keep_mask(B: int, H: int, N: int, p_drop: float, seed: int, offset: int = 0,
+                      lib=None):
+    """Keep mask z [B,H,N,N] (bool; row = query, column = key) of the dropout forward."""
+    lib = lib or load()
+    m = np.empty((B, H, N, N), np.uint8)
+    _check(lib.oracle_dropout_keep_mask(B, H, N, float(p_drop), int(seed), int(offset), _ptr(m)),
+           "oracle_dropout_keep_mask")
+    return m.astype(bool)
 
 
 def softmax_partial(s, Vblk, lib=None):

@@ -48,6 +48,21 @@
  *           and contributes nothing to any gradient.  Equivalently: batch b is
  *           [STD] on its first seqlens[b] tokens.  seqlens = NULL: all N.
  *
+ *   [DROP]  downcodes.com "triton transformer", usage section: the
+ *           `attn_dropout = 0.1` option (attention dropout).  The page gives
+ *           no formula; reading: inverted dropout on the normalised
+ *           probabilities, O_i = sum_j P_ij z_ij / (1 - p) v_j with z_ij in
+ *           {0, 1} kept with probability 1 - p; LSE is that of the undropped
+ *           scores.  The page gives no random-number convention either:
+ *           z_ij comes from the counter-based generator Philox-4x32-10
+ *           (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as
+ *           1, 2, 3", SC'11), called with
+ *             counter = (j / 4, i, b * H + h, offset), key = (seed mod 2^32,
+ *                       seed / 2^32)
+ *           and z_ij = 1 iff word (j mod 4) of the output is below
+ *           floor((1 - p) 2^32), for query i, key j of query head h of
+ *           batch b (positions counted from the start of the sequence).
+ *
  * Every function returns 0 on success, -1 on a bad argument, -2 if memory
  * could not be allocated.
  */
@@ -95,6 +110,81 @@ static int bad_seqlens(const int32_t *seqlens, int64_t B, int64_t N)
     return 0;
 }
 
+/*
+ * [DROP] Philox-4x32 with 10 rounds, as the SC'11 paper defines it: each
+ * round multiplies counter words 0 and 2 by the constants M0, M1 into 64-bit
+ * products (hi, lo), and the new counter is
+ *     (hi(M1 c2) ^ c1 ^ k0,  lo(M1 c2),  hi(M0 c0) ^ c3 ^ k1,  lo(M0 c0));
+ * between rounds the key is bumped by the Weyl constants W0, W1.
+ */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+    const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = (uint64_t)M0 * c0, p1 = (uint64_t)M1 * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
+        c0 = n0;
+        c2 = n2;
+        k0 += W0;
+        k1 += W1;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+/* [DROP] parameters; NULL or p == 0 means no dropout. */
+struct dropout {
+    double p;            /* probability of dropping, [0, 1) */
+    uint32_t key[2];     /* the seed */
+    uint32_t offset;     /* counter word 3 */
+    uint64_t threshold;  /* floor((1 - p) 2^32): keep iff word < threshold */
+    double keep_scale;   /* 1 / (1 - p) */
+};
+
+static int make_dropout(struct dropout *dr, double p, uint64_t seed, uint32_t offset)
+{
+    if (!(p >= 0.0 && p < 1.0))
+        return -1;
+    dr->p = p;
+    dr->key[0] = (uint32_t)seed;
+    dr->key[1] = (uint32_t)(seed >> 32);
+    dr->offset = offset;
+    dr->threshold = (uint64_t)floor((1.0 - p) * 4294967296.0);
+    dr->keep_scale = 1.0 / (1.0 - p);
+    return 0;
+}
+
+/* z_ij of [DROP] for query i, key j of query head bh = b * H + h. */
+static int dropout_keep(const struct dropout *dr, int64_t bh, int64_t i, int64_t j)
+{
+    const uint32_t ctr[4] = {(uint32_t)(j / 4), (uint32_t)i, (uint32_t)bh, dr->offset};
+    uint32_t w[4];
+    oracle_philox4x32_10(ctr, dr->key, w);
+    return (uint64_t)w[j % 4] < dr->threshold;
+}
+
+/* The [DROP] keep mask z as bytes [B, H, N, N] (row = query, column = key). */
+int oracle_dropout_keep_mask(int64_t B, int64_t H, int64_t N, double p, uint64_t seed,
+                             uint32_t offset, uint8_t *mask)
+{
+    struct dropout dr;
+    if (!mask || B < 1 || H < 1 || N < 1 || make_dropout(&dr, p, seed, offset))
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < B * H * N; ++r)
+        for (int64_t j = 0; j < N; ++j)
+            mask[r * N + j] = (uint8_t)dropout_keep(&dr, r / N, r % N, j);
+    return 0;
+}
+
 /* [GQA]: key/value head of query head bh = b * H + h. */
 static int64_t kv_head(int64_t bh, int64_t H, int64_t Hkv)
 {
@@ -108,13 +198,14 @@ static int64_t kv_head(int64_t bh, int64_t H, int64_t Hkv)
  *   m     = max_j s_j                    ([SAFE])
  *   LSE_i = m + ln sum_j exp(s_j - m)
  *   P_j   = exp(s_j - m) / sum_j exp(s_j - m)
- *   O_i   = sum_j P_j v_j
- * s is caller-provided scratch of N doubles.
+ *   O_i   = sum_j P_j v_j                (sum_j P_j z_ij / (1 - p) v_j with [DROP])
+ * s is caller-provided scratch of N doubles; bh names the query head for
+ * [DROP] (dr = NULL: no dropout).
  */
 static void attention_row(const void *Q, const void *K, const void *V, int dtype,
                           int64_t n_keys, int64_t d, int64_t q_base, int64_t kv_base, int64_t i,
-                          double scale, int causal, double *s,
-                          double *o_row, double *lse)
+                          double scale, int causal, const struct dropout *dr, int64_t bh,
+                          double *s, double *o_row, double *lse)
 {
     const int64_t N = n_keys;
     for (int64_t j = 0; j < N; ++j) {
@@ -139,7 +230,9 @@ static void attention_row(const void *Q, const void *K, const void *V, int dtype
     for (int64_t c = 0; c < d; ++c)
         o_row[c] = 0.0;
     for (int64_t j = 0; j < N; ++j) {
-        const double p = s[j] / sum;
+        double p = s[j] / sum;
+        if (dr)
+            p = dropout_keep(dr, bh, i, j) ? p * dr->keep_scale : 0.0;
         if (p == 0.0)
             continue;
         for (int64_t c = 0; c < d; ++c)
@@ -147,16 +240,21 @@ static void attention_row(const void *Q, const void *K, const void *V, int dtype
     }
 }
 
-/* Full forward with [GQA] heads and [PAD] lengths: O [B,H,N,d] and LSE
- * [B,H,N], both double; K, V are [B,Hkv,N,d]; seqlens [B] or NULL. */
-int oracle_attention_forward_varlen(const void *Q, const void *K, const void *V, int dtype,
-                                    const int32_t *seqlens, int64_t B, int64_t H, int64_t Hkv,
-                                    int64_t N, int64_t d, double scale, int causal,
-                                    double *O, double *LSE)
+/* Full forward with [GQA] heads, [PAD] lengths and [DROP] dropout: O
+ * [B,H,N,d] and LSE [B,H,N], both double; K, V are [B,Hkv,N,d]; seqlens [B]
+ * or NULL; p_drop = 0: no dropout. */
+int oracle_attention_forward_dropout(const void *Q, const void *K, const void *V, int dtype,
+                                     const int32_t *seqlens, int64_t B, int64_t H, int64_t Hkv,
+                                     int64_t N, int64_t d, double scale, int causal,
+                                     double p_drop, uint64_t seed, uint32_t offset,
+                                     double *O, double *LSE)
 {
+    struct dropout drop;
     if (!Q || !K || !V || !O || !LSE || bad_shape(B, H, N, d, dtype) ||
-        Hkv < 1 || Hkv > H || H % Hkv != 0 || bad_seqlens(seqlens, B, N))
+        Hkv < 1 || Hkv > H || H % Hkv != 0 || bad_seqlens(seqlens, B, N) ||
+        make_dropout(&drop, p_drop, seed, offset))
         return -1;
+    const struct dropout *dr = p_drop > 0.0 ? &drop : NULL;
     const int64_t rows = B * H * N;
     int failed = 0;
 #pragma omp parallel
@@ -179,11 +277,21 @@ int oracle_attention_forward_varlen(const void *Q, const void *K, const void *V,
                 continue;
             }
             attention_row(Q, K, V, dtype, len, d, bh * N * d, kv_head(bh, H, Hkv) * N * d, i,
-                          scale, causal, s, O + r * d, LSE + r);
+                          scale, causal, dr, bh, s, O + r * d, LSE + r);
         }
         free(s);
     }
     return failed ? -2 : 0;
+}
+
+/* Full forward with [GQA] heads and [PAD] lengths, no dropout. */
+int oracle_attention_forward_varlen(const void *Q, const void *K, const void *V, int dtype,
+                                    const int32_t *seqlens, int64_t B, int64_t H, int64_t Hkv,
+                                    int64_t N, int64_t d, double scale, int causal,
+                                    double *O, double *LSE)
+{
+    return oracle_attention_forward_dropout(Q, K, V, dtype, seqlens, B, H, Hkv, N, d, scale,
+                                            causal, 0.0, 0, 0, O, LSE);
 }
 
 /* Full forward with [GQA] heads, no padding. */
@@ -234,8 +342,8 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
             if (!s)
                 continue;
             const int64_t bh = rows[k] / N, i = rows[k] % N;
-            attention_row(Q, K, V, dtype, N, d, bh * N * d, bh * N * d, i, scale, causal, s,
-                          O_rows + k * d, LSE_rows + k);
+            attention_row(Q, K, V, dtype, N, d, bh * N * d, bh * N * d, i, scale, causal, NULL,
+                          bh, s, O_rows + k * d, LSE_rows + k);
         }
         free(s);
     }
@@ -257,23 +365,33 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
  * With [GQA] heads the key/value gradients of a key/value head are the sums
  * of these over the query heads that share it.  With [PAD] lengths each
  * (batch, head) is the same on its first len tokens (P = 0 outside) and all
- * gradients of padding tokens are 0.  dQ is double [B,H,N,d]; dK, dV are
- * double [B,Hkv,N,d].
+ * gradients of padding tokens are 0.  With [DROP] the output is
+ * O_i = sum_j Pd_ij v_j, Pd_ij = P_ij z_ij / (1 - p), and by the chain rule
+ *   dV_j  = sum_i Pd_ij dO_i
+ *   dP_ij = <dO_i, v_j> z_ij / (1 - p)       (gradient with respect to P)
+ * with D, dS, dQ, dK as above (D_i = sum_j P_ij dP_ij still equals
+ * <dO_i, O_i>).  dQ is double [B,H,N,d]; dK, dV are double [B,Hkv,N,d].
  */
-int oracle_attention_backward_varlen(const void *Q, const void *K, const void *V,
-                                     const void *dO, int dtype, const int32_t *seqlens,
-                                     int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
-                                     double scale, int causal,
-                                     double *dQ, double *dK, double *dV)
+int oracle_attention_backward_dropout(const void *Q, const void *K, const void *V,
+                                      const void *dO, int dtype, const int32_t *seqlens,
+                                      int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                      double scale, int causal, double p_drop, uint64_t seed,
+                                      uint32_t offset, double *dQ, double *dK, double *dV)
 {
+    struct dropout drop;
     if (!Q || !K || !V || !dO || !dQ || !dK || !dV || bad_shape(B, H, N, d, dtype) ||
-        Hkv < 1 || Hkv > H || H % Hkv != 0 || bad_seqlens(seqlens, B, N))
+        Hkv < 1 || Hkv > H || H % Hkv != 0 || bad_seqlens(seqlens, B, N) ||
+        make_dropout(&drop, p_drop, seed, offset))
         return -1;
+    const struct dropout *dr = p_drop > 0.0 ? &drop : NULL;
     double *P = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
     double *dS = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
-    if (!P || !dS) {
+    /* z_ij / (1 - p) of the current head (only with dropout) */
+    double *Z = dr ? (double *)malloc((size_t)N * (size_t)N * sizeof(double)) : NULL;
+    if (!P || !dS || (dr && !Z)) {
         free(P);
         free(dS);
+        free(Z);
         return -2;
     }
     for (int64_t e = 0; e < B * Hkv * N * d; ++e) {
@@ -311,6 +429,9 @@ int oracle_attention_backward_varlen(const void *Q, const void *K, const void *V
             }
             for (int64_t j = 0; j < N; ++j)
                 s[j] /= sum;
+            if (dr)
+                for (int64_t j = 0; j < N; ++j)
+                    Z[i * N + j] = dropout_keep(dr, bh, i, j) ? dr->keep_scale : 0.0;
         }
         /* dP, D and dS. */
 #pragma omp parallel for schedule(dynamic, 8)
@@ -320,7 +441,7 @@ int oracle_attention_backward_varlen(const void *Q, const void *K, const void *V
                 double acc = 0.0;
                 for (int64_t c = 0; c < d; ++c)
                     acc += ld(dO, base + i * d + c, dtype) * ld(V, kv_base + j * d + c, dtype);
-                ds[j] = acc; /* dP_ij */
+                ds[j] = dr ? acc * Z[i * N + j] : acc; /* dP_ij */
             }
             double D = 0.0;
             for (int64_t j = 0; j < N; ++j)
@@ -344,8 +465,9 @@ int oracle_attention_backward_varlen(const void *Q, const void *K, const void *V
             for (int64_t c = 0; c < d; ++c) {
                 double acc_k = 0.0, acc_v = 0.0;
                 for (int64_t i = 0; i < N; ++i) {
+                    const double pd = dr ? P[i * N + j] * Z[i * N + j] : P[i * N + j];
                     acc_k += dS[i * N + j] * ld(Q, base + i * d + c, dtype);
-                    acc_v += P[i * N + j] * ld(dO, base + i * d + c, dtype);
+                    acc_v += pd * ld(dO, base + i * d + c, dtype);
                 }
                 dK[kv_base + j * d + c] += scale * acc_k;
                 dV[kv_base + j * d + c] += acc_v;
@@ -354,7 +476,19 @@ int oracle_attention_backward_varlen(const void *Q, const void *K, const void *V
     }
     free(P);
     free(dS);
+    free(Z);
     return 0;
+}
+
+/* Backward with [GQA] heads and [PAD] lengths, no dropout. */
+int oracle_attention_backward_varlen(const void *Q, const void *K, const void *V,
+                                     const void *dO, int dtype, const int32_t *seqlens,
+                                     int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                     double scale, int causal,
+                                     double *dQ, double *dK, double *dV)
+{
+    return oracle_attention_backward_dropout(Q, K, V, dO, dtype, seqlens, B, H, Hkv, N, d, scale,
+                                             causal, 0.0, 0, 0, dQ, dK, dV);
 }
 
 /* Backward with [GQA] heads, no padding. */

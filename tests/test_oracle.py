@@ -465,6 +465,138 @@ def pin_padding_backward_vs_autograd(lib):
         _close(dV, tv.grad.numpy())
 
 
+# ----------------------------------------------------------------------------
+# Dropout pins (downcodes.com "triton transformer", usage section:
+# attn_dropout).  The generator is Philox-4x32-10 (Salmon, Moraes, Dror,
+# Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11).
+# ----------------------------------------------------------------------------
+
+# Known-answer vectors published with the generator (Random123 distribution,
+# kat_vectors, philox4x32 with 10 rounds): (counter, key, output).
+PHILOX_KAT = [
+    ((0, 0, 0, 0), (0, 0), (0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8)),
+    ((0xFFFFFFFF,) * 4, (0xFFFFFFFF,) * 2, (0x408F276D, 0x41C83B0E, 0xA20BC7C6, 0x6D5451FD)),
+    ((0x243F6A88, 0x85A308D3, 0x13198A2E, 0x03707344), (0xA4093822, 0x299F31D0),
+     (0xD16CFE09, 0x94FDCCEB, 0x5001E420, 0x24126EA1)),
+]
+
+
+def _philox_py(ctr, key, rounds=10):
+    """Philox-4x32 written out from the SC'11 definition (independent of the C)."""
+    c, k = list(ctr), list(key)
+    for _ in range(rounds):
+        a, b = 0xD2511F53 * c[0], 0xCD9E8D57 * c[2]
+        c = [((b >> 32) ^ c[1] ^ k[0]) & 0xFFFFFFFF, b & 0xFFFFFFFF,
+             ((a >> 32) ^ c[3] ^ k[1]) & 0xFFFFFFFF, a & 0xFFFFFFFF]
+        k = [(k[0] + 0x9E3779B9) & 0xFFFFFFFF, (k[1] + 0xBB67AE85) & 0xFFFFFFFF]
+    return tuple(c)
+
+
+def pin_philox_known_answers(lib):
+    for ctr, key, want in PHILOX_KAT:
+        assert _philox_py(ctr, key) == want
+        assert tuple(int(x) for x in oracle.philox4x32_10(ctr, key, lib=lib)) == want
+
+
+def pin_dropout_mask_convention(lib):
+    """Keep mask = the stated counter layout (j/4, i, b*H+h, offset), key =
+    seed halves, word j%4 below floor((1-p) 2^32), evaluated independently."""
+    assert _philox_py(*PHILOX_KAT[2][:2]) == PHILOX_KAT[2][2]
+    B, H, N, p, seed, offset = 2, 3, 11, 0.3, 0x0123456789ABCDEF, 7
+    m = oracle.dropout_keep_mask(B, H, N, p, seed, offset, lib=lib)
+    t = math.floor((1.0 - p) * 2.0 ** 32)
+    key = (seed & 0xFFFFFFFF, seed >> 32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(N):
+                for j in range(N):
+                    w = _philox_py((j // 4, i, b * H + h, offset), key)[j % 4]
+                    assert m[b, h, i, j] == (w < t), (b, h, i, j)
+
+
+def pin_dropout_keep_rate(lib):
+    """Each element is kept with probability 1 - p: the kept fraction of 2^20
+    draws is within 6 standard deviations; p = 0 keeps everything."""
+    for p in (0.1, 0.5, 0.9):
+        m = oracle.dropout_keep_mask(1, 4, 512, p, 99, 3, lib=lib)
+        n = m.size
+        assert abs(m.mean() - (1 - p)) <= 6 * math.sqrt(p * (1 - p) / n), (p, m.mean())
+    assert oracle.dropout_keep_mask(1, 1, 64, 0.0, 5, lib=lib).all()
+
+
+def pin_dropout_zero_is_plain_attention(lib):
+    r = _rng(31)
+    Q, K, V = (r.standard_normal((2, 2, 9, 4)) for _ in range(3))
+    O0, L0 = oracle.attention_forward(Q, K, V, 0.5, True, lib=lib)
+    O, L = oracle.attention_forward_dropout(Q, K, V, 0.5, True, 0.0, 1234, lib=lib)
+    assert np.array_equal(O, O0) and np.array_equal(L, L0)
+
+
+def _dropout_torch(Q, K, V, z, p, scale, causal, seqlens):
+    """(softmax(scale Q K^T, masked) * z / (1 - p)) V in fp64 torch, with grads."""
+    B, H, N, _ = Q.shape
+    G = H // K.shape[1]
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+    mask = _key_mask(seqlens if seqlens is not None else [N] * B, N, causal)
+    s = (scale * tq @ tk.repeat_interleave(G, dim=1).transpose(-1, -2)).masked_fill(
+        ~mask, float("-inf"))
+    P = torch.softmax(s, dim=-1)
+    out = (P * torch.from_numpy(z.astype(np.float64)) / (1.0 - p)) @ tv.repeat_interleave(G, dim=1)
+    return out, torch.logsumexp(s, dim=-1), (tq, tk, tv)
+
+
+DROPOUT_CASES = [(2, 2, 1, 9, 4, True, [9, 6], 0.25), (1, 3, 3, 13, 8, False, None, 0.6),
+                 (1, 4, 2, 10, 4, False, [7], 0.1)]
+
+
+def pin_dropout_forward_vs_torch(lib):
+    """O equals the explicit formula with the mask; LSE is the undropped one."""
+    r = _rng(32)
+    for (B, H, Hkv, N, d, causal, sl, p) in DROPOUT_CASES:
+        Q = r.standard_normal((B, H, N, d))
+        K, V = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+        seed, offset = 1000 + N, 5
+        O, LSE = oracle.attention_forward_dropout(Q, K, V, 0.7, causal, p, seed, offset,
+                                                  seqlens=sl, lib=lib)
+        z = oracle.dropout_keep_mask(B, H, N, p, seed, offset, lib=lib)
+        assert 0 < z.mean() < 1
+        ref, lse, _ = _dropout_torch(Q, K, V, z, p, 0.7, causal, sl)
+        for b in range(B):
+            n = N if sl is None else sl[b]
+            _close(O[b, :, :n], ref[b, :, :n].detach().numpy())
+            _close(LSE[b, :, :n], lse[b, :, :n].detach().numpy())
+
+
+def pin_dropout_backward_vs_autograd(lib):
+    r = _rng(33)
+    for (B, H, Hkv, N, d, causal, sl, p) in DROPOUT_CASES:
+        Q, dO = (r.standard_normal((B, H, N, d)) for _ in range(2))
+        K, V = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+        seed, offset = 77 + N, 2
+        z = oracle.dropout_keep_mask(B, H, N, p, seed, offset, lib=lib)
+        out, _, (tq, tk, tv) = _dropout_torch(Q, K, V, z, p, 0.7, causal, sl)
+        lens = [N] * B if sl is None else sl
+        real = (torch.arange(N)[None, :] < torch.tensor(lens)[:, None])[:, None, :, None]
+        (out * torch.from_numpy(dO) * real).sum().backward()
+        dQ, dK, dV = oracle.attention_backward_dropout(Q, K, V, dO, 0.7, causal, p, seed, offset,
+                                                       seqlens=sl, lib=lib)
+        _close(dQ, (tq.grad * real).numpy())
+        _close(dK, tk.grad.numpy())
+        _close(dV, tv.grad.numpy())
+
+
+def pin_dropout_is_unbiased(lib):
+    """Inverted dropout leaves O unchanged in expectation: the mean over 1500
+    seeds is within 6 standard errors of the undropped O."""
+    r = _rng(34)
+    Q, K, V = (r.standard_normal((1, 1, 6, 3)) for _ in range(3))
+    O0, _ = oracle.attention_forward(Q, K, V, 0.8, False, lib=lib)
+    runs = np.stack([oracle.attention_forward_dropout(Q, K, V, 0.8, False, 0.4, sd, lib=lib)[0]
+                     for sd in range(1500)])
+    se = runs.std(axis=0) / math.sqrt(len(runs))
+    assert np.all(np.abs(runs.mean(axis=0) - O0) <= 6 * se + 1e-12)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -481,6 +613,11 @@ def test_bad_arguments_are_rejected():
     Q = np.zeros((1, 1, 3, 4))
     with pytest.raises(RuntimeError):
         oracle.attention_forward_rows(Q, Q, Q, 1.0, False, np.array([3]), lib=lib)
+    for p in (1.0, -0.1, float("nan")):
+        with pytest.raises(RuntimeError):
+            oracle.attention_forward_dropout(Q, Q, Q, 1.0, False, p, 1, lib=lib)
+        with pytest.raises(RuntimeError):
+            oracle.dropout_keep_mask(1, 1, 3, p, 1, lib=lib)
 
 
 def test_golden_regression():
@@ -513,7 +650,7 @@ MUTANTS = {
     "causal_off_by_one": ("if (causal && j > i)", "if (causal && j >= i)", 0),
     "causal_flipped": ("if (causal && j > i)", "if (causal && j < i)", 0),
     "lse_missing_max": ("*lse = m + log(sum);", "*lse = log(sum);", 0),
-    "no_normalisation": ("const double p = s[j] / sum;", "const double p = s[j];", 0),
+    "no_normalisation": ("double p = s[j] / sum;", "double p = s[j];", 0),
     "wrong_value_row": ("o_row[c] += p * ld(V, kv_base + j * d + c, dtype);",
                         "o_row[c] += p * ld(V, kv_base + i * d + c, dtype);", 0),
     "gqa_interleaved_heads": ("return (bh / H) * Hkv + (bh % H) / (H / Hkv);",
@@ -529,13 +666,27 @@ MUTANTS = {
     "exp_sign": ("s[j] = exp(s[j] - m); /* exp(-inf)", "s[j] = exp(m - s[j]); /* exp(-inf)", 0),
     "bwd_drop_scale_in_scores": ("s[j] = scale * acc;", "s[j] = acc;", 1),
     "bwd_drop_D": ("ds[j] = P[i * N + j] * (ds[j] - D);", "ds[j] = P[i * N + j] * ds[j];", 0),
-    "bwd_dV_uses_dS": ("acc_v += P[i * N + j] * ld(dO", "acc_v += dS[i * N + j] * ld(dO", 0),
+    "bwd_dV_uses_dS": ("acc_v += pd * ld(dO", "acc_v += dS[i * N + j] * ld(dO", 0),
     "bwd_dQ_no_scale": ("dQ[base + i * d + c] = scale * acc;", "dQ[base + i * d + c] = acc;", 0),
     "bwd_dK_transposed_dS": ("acc_k += dS[i * N + j]", "acc_k += dS[j * N + i]", 0),
     "bwd_causal_off_by_one": ("if (causal && j > i)", "if (causal && j >= i)", 1),
     "merge_unweighted": ("o[c] = (a * o_x[c] + b * o_y[c]) / ll;",
                          "o[c] = (exp(m_x - mm) * o_x[c] + exp(m_y - mm) * o_y[c]) / ll;", 0),
     "merge_max_wrong": ("const double mm = fmax(m_x, m_y);", "const double mm = m_x;", 0),
+    "philox_seven_rounds": ("for (int r = 0; r < 10; ++r) {", "for (int r = 0; r < 7; ++r) {", 0),
+    "philox_hi_lo_swapped": ("c1 = (uint32_t)p1;", "c1 = (uint32_t)(p1 >> 32);", 0),
+    "drop_counter_transposed": ("{(uint32_t)(j / 4), (uint32_t)i,", "{(uint32_t)(i / 4), (uint32_t)j,", 0),
+    "drop_word_index": ("return (uint64_t)w[j % 4] <", "return (uint64_t)w[i % 4] <", 0),
+    "drop_keep_inverted": ("return (uint64_t)w[j % 4] < dr->threshold;",
+                           "return (uint64_t)w[j % 4] >= dr->threshold;", 0),
+    "drop_seed_halves_swapped": ("dr->key[0] = (uint32_t)seed;", "dr->key[0] = (uint32_t)(seed >> 32);", 0),
+    "drop_no_keep_scale": ("? p * dr->keep_scale : 0.0;", "? p : 0.0;", 0),
+    "drop_fwd_kv_head": ("scale, causal, dr, bh, s,", "scale, causal, dr, kv_head(bh, H, Hkv), s,", 0),
+    "drop_bwd_dP_unmasked": ("ds[j] = dr ? acc * Z[i * N + j] : acc;", "ds[j] = acc;", 0),
+    "drop_bwd_dV_undropped": ("const double pd = dr ? P[i * N + j] * Z[i * N + j] : P[i * N + j];",
+                              "const double pd = P[i * N + j];", 0),
+    "drop_bwd_kv_head": ("Z[i * N + j] = dropout_keep(dr, bh, i, j)",
+                         "Z[i * N + j] = dropout_keep(dr, kv_head(bh, H, Hkv), i, j)", 0),
 }
 
 
