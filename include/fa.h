@@ -89,6 +89,30 @@ fa_status fa_forward_varlen(const void *Q, const void *K, const void *V, void *O
                             float scale, int causal, cudaStream_t stream);
 
 /*
+ * Attention dropout (the attn_dropout option of downcodes.com "triton
+ * transformer", usage section; the page gives no formula).  Inverted dropout
+ * on the normalised probabilities:
+ *     O_i = sum_j P_ij z_ij / (1 - dropout_p) v_j,   LSE as without dropout
+ * with the keep bit z_ij of query i, key j of query head bh = b * H + h taken
+ * from the counter-based generator Philox-4x32-10 (Salmon et al., "Parallel
+ * Random Numbers: As Easy as 1, 2, 3", SC'11):
+ *     w = Philox(counter = (j / 4, i, bh, offset), key = (seed & 0xffffffff, seed >> 32))
+ *     z_ij = (w[j % 4] < floor((1 - dropout_p) * 2^32))
+ * (i, j counted from the start of the sequence).  The same (seed, offset)
+ * given to fa_backward_dropout regenerates the mask; a caller that needs a
+ * fresh mask per call changes either.
+ *   dropout_p : in [0, 1) (FA_ERR_INVALID_ARG otherwise, NaN included);
+ *               0 -- or any value with floor((1 - p) 2^32) = 2^32 -- is
+ *               exactly fa_forward_varlen.
+ * Other arguments as fa_forward_varlen (seqlens may be NULL; K/V with H_kv
+ * heads).  The keep-bit generation costs integer work in the softmax warps.
+ */
+fa_status fa_forward_dropout(const void *Q, const void *K, const void *V, void *O, float *LSE,
+                             const int *seqlens, int B, int H, int H_kv, int N, int d,
+                             float scale, int causal, float dropout_p, unsigned long long seed,
+                             unsigned int offset, cudaStream_t stream);
+
+/*
  * FP8 forward (the FlashAttention-3 direction of the pages: FP8 compute,
  * systems-analysis.info "FlashAttention-2 (VI)", FlashAttention-3 section).
  *   Q8, K8, V8 : [B,H,N,d] / [B,H_kv,N,d] E4M3 bytes (__nv_fp8_e4m3); the
@@ -153,6 +177,20 @@ fa_status fa_backward_varlen(const void *Q, const void *K, const void *V, const 
                              void *workspace, size_t workspace_bytes, const int *seqlens,
                              int B, int H, int H_kv, int N, int d, float scale, int causal,
                              cudaStream_t stream);
+
+/*
+ * Backward of fa_forward_dropout: the same (dropout_p, seed, offset) and
+ * seqlens as the forward call that produced O and LSE.  With
+ * Pd_ij = P_ij z_ij / (1 - p):  dV_j = sum_i Pd_ij dO_i,
+ * dS_ij = P_ij (z_ij <dO_i, v_j> / (1 - p) - <dO_i, O_i>), dQ and dK from dS
+ * as in fa_backward.  Other arguments as fa_backward_varlen.
+ */
+fa_status fa_backward_dropout(const void *Q, const void *K, const void *V, const void *O,
+                              const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
+                              void *workspace, size_t workspace_bytes, const int *seqlens,
+                              int B, int H, int H_kv, int N, int d, float scale, int causal,
+                              float dropout_p, unsigned long long seed, unsigned int offset,
+                              cudaStream_t stream);
 
 /*
  * Size of the device array fa_backward_noalloc uses as its workspace (64 MiB).

@@ -18,9 +18,10 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 
 # Every entry point include/fa.h declares.
-EXPORTS = ("fa_forward", "fa_forward_gqa", "fa_forward_varlen", "fa_forward_fp8",
-           "fa_backward_workspace_bytes",
-           "fa_backward", "fa_backward_gqa", "fa_backward_varlen", "fa_backward_noalloc",
+EXPORTS = ("fa_forward", "fa_forward_gqa", "fa_forward_varlen", "fa_forward_dropout",
+           "fa_forward_fp8", "fa_backward_workspace_bytes",
+           "fa_backward", "fa_backward_gqa", "fa_backward_varlen", "fa_backward_dropout",
+           "fa_backward_noalloc",
            "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_str", "fa_version")
 
 # Size of the library's built-in workspace used by fa_backward_noalloc.
@@ -62,6 +63,13 @@ def load_library(path: str | None = None):
     lib.fa_backward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, i, i, i, i,
                                        i, f, i, vp]
     lib.fa_backward_varlen.restype = i
+    u64, u32 = ctypes.c_ulonglong, ctypes.c_uint
+    lib.fa_forward_dropout.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, f, u64, u32,
+                                       vp]
+    lib.fa_forward_dropout.restype = i
+    lib.fa_backward_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, i, i, i, i,
+                                        i, f, i, f, u64, u32, vp]
+    lib.fa_backward_dropout.restype = i
     lib.fa_forward_fp8.argtypes = [vp, vp, vp, vp, vp, f, f, f, i, i, i, i, i, f, i, vp]
     lib.fa_forward_fp8.restype = i
     lib.fa_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
@@ -130,10 +138,12 @@ def _seqlens_ptr(seqlens, B, device):
 
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
             scale: float | None = None, out: torch.Tensor | None = None,
-            lse: torch.Tensor | None = None, stream=None, seqlens: torch.Tensor | None = None):
+            lse: torch.Tensor | None = None, stream=None, seqlens: torch.Tensor | None = None,
+            dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
     """O, LSE = softmax(scale Q K^T [+causal]) V and its per-row logsumexp.
     K and V may have fewer heads than Q (grouped-/multi-query attention);
-    seqlens [B] marks tokens >= seqlens[b] of batch b as padding."""
+    seqlens [B] marks tokens >= seqlens[b] of batch b as padding; dropout_p > 0
+    applies attention dropout with the Philox keep mask of (seed, offset)."""
     B, H, N, d, Hkv = _check_kv_heads(q, k, v)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
@@ -142,9 +152,16 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Fa
     if l.dtype != torch.float32 or not l.is_contiguous() or tuple(l.shape) != (B, H, N):
         raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
     keep, sl = _seqlens_ptr(seqlens, B, q.device)
-    st = load_library().fa_forward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                          l.data_ptr(), sl, B, H, Hkv, N, d, scale,
-                                          int(bool(causal)), _stream_handle(stream))
+    lib = load_library()
+    if dropout_p:
+        st = lib.fa_forward_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    l.data_ptr(), sl, B, H, Hkv, N, d, scale, int(bool(causal)),
+                                    float(dropout_p), int(seed), int(offset),
+                                    _stream_handle(stream))
+    else:
+        st = lib.fa_forward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   l.data_ptr(), sl, B, H, Hkv, N, d, scale, int(bool(causal)),
+                                   _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_forward")
     return o, l
@@ -176,9 +193,11 @@ def forward_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float
 
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, stream=None,
-             seqlens: torch.Tensor | None = None):
+             seqlens: torch.Tensor | None = None, dropout_p: float = 0.0, seed: int = 0,
+             offset: int = 0):
     """dQ, dK, dV of <O, dO> (scores recomputed from the saved LSE).  With K/V
-    of fewer heads, dK/dV are summed over each group of query heads."""
+    of fewer heads, dK/dV are summed over each group of query heads.  The
+    dropout arguments must be those of the forward call."""
     B, H, N, d, Hkv = _check_kv_heads(q, k, v)
     _check_qkv(q, o, do)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -190,11 +209,15 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     keep, sl = _seqlens_ptr(seqlens, B, q.device)
-    st = lib.fa_backward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                                dv.data_ptr(), workspace.data_ptr(),
-                                workspace.numel() * workspace.element_size(), sl,
-                                B, H, Hkv, N, d, scale, int(bool(causal)), _stream_handle(stream))
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+            lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), sl, B, H, Hkv, N, d, scale,
+            int(bool(causal)))
+    if dropout_p:
+        st = lib.fa_backward_dropout(*args, float(dropout_p), int(seed), int(offset),
+                                     _stream_handle(stream))
+    else:
+        st = lib.fa_backward_varlen(*args, _stream_handle(stream))
     if st != FA_OK:
         raise FaError(st, "fa_backward")
     return dq, dk, dv
@@ -217,20 +240,29 @@ def selftest_bounded_wait(timeout_ns: int = 20_000_000, stream=None) -> tuple[in
 
 class _Attention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, causal, scale):
-        o, lse = forward(q, k, v, causal=causal, scale=scale)
+    def forward(ctx, q, k, v, causal, scale, dropout_p, seed, offset):
+        o, lse = forward(q, k, v, causal=causal, scale=scale, dropout_p=dropout_p, seed=seed,
+                         offset=offset)
         ctx.save_for_backward(q, k, v, o, lse)
         ctx.causal, ctx.scale = causal, scale
+        ctx.dropout = (dropout_p, seed, offset)
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
+        p, seed, offset = ctx.dropout
         dq, dk, dv = backward(q, k, v, o, do.contiguous(), lse, causal=ctx.causal,
-                              scale=ctx.scale)
-        return dq, dk, dv, None, None
+                              scale=ctx.scale, dropout_p=p, seed=seed, offset=offset)
+        return dq, dk, dv, None, None, None, None, None
 
 
-def attention(q, k, v, causal: bool = False, scale: float | None = None):
-    """Differentiable exact attention (autograd wrapper over forward/backward)."""
-    return _Attention.apply(q, k, v, causal, scale)
+def attention(q, k, v, causal: bool = False, scale: float | None = None, dropout_p: float = 0.0,
+              seed: int | None = None, offset: int = 0):
+    """Differentiable exact attention (autograd wrapper over forward/backward).
+    With dropout_p > 0 and no seed, a seed is drawn from torch's default CPU
+    generator, so torch.manual_seed makes the mask reproducible; the backward
+    regenerates the same mask."""
+    if dropout_p and seed is None:
+        seed = int(torch.randint(0, 2 ** 62, (1,)).item())
+    return _Attention.apply(q, k, v, causal, scale, float(dropout_p), int(seed or 0), int(offset))

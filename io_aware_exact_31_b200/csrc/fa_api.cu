@@ -23,8 +23,9 @@ struct DeviceState {
     bool checked = false;
     bool supported = false;
     uint32_t* err = nullptr;  // device address of g_err_word on this device
-    bool fwd_attr[3] = {false, false, false};  // d = 64, d = 128, d = 128 E4M3
-    bool bwd_attr[2] = {false, false};
+    // d = 64, d = 128, d = 128 E4M3, d = 64 dropout, d = 128 dropout
+    bool fwd_attr[5] = {false, false, false, false, false};
+    bool bwd_attr[4] = {false, false, false, false};  // d = 64, 128; then with dropout
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -84,13 +85,29 @@ fa_status check_heads(int H, int Hkv) {
     return FA_OK;
 }
 
+// Attention-dropout parameters from (p, seed, offset).  *on = false when p
+// is so small that 1 - p rounds to 1 (floor((1 - p) 2^32) = 2^32: nothing is
+// ever dropped), which runs the kernels without dropout.
+fa_status make_dropout(float p, uint64_t seed, uint32_t offset, DropoutParams* d, bool* on) {
+    if (!(p >= 0.f && p < 1.f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
+    const double t = std::floor((1.0 - static_cast<double>(p)) * 4294967296.0);
+    *on = t < 4294967296.0;
+    d->seed_lo = static_cast<uint32_t>(seed);
+    d->seed_hi = static_cast<uint32_t>(seed >> 32);
+    d->offset = offset;
+    d->threshold = *on ? static_cast<uint32_t>(t) : 0xFFFFFFFFu;
+    d->keep_scale = static_cast<float>(1.0 / (1.0 - static_cast<double>(p)));
+    return FA_OK;
+}
+
 // scale_qk multiplies the scores (dequant scales of E4M3 Q and K), scale_v
-// the output (dequant scale of E4M3 V); both 1 for bf16 inputs.
-template <int D, bool F8>
+// the output (dequant scale of E4M3 V); both 1 for bf16 inputs.  DROP: drop
+// holds the dropout parameters.
+template <int D, bool F8, bool DROP = false>
 fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const void* V, void* O,
                          float* LSE, int B, int H, int Hkv, int N, const int* seqlens,
                          float scale, int causal, cudaStream_t stream, double scale_qk = 1.0,
-                         float scale_v = 1.f) {
+                         float scale_v = 1.f, const DropoutParams* drop = nullptr) {
     using C = FwdCfg<D, F8>;
     CUtensorMap mq, mk, mv;
     const uint64_t depth = static_cast<uint64_t>(B) * H;
@@ -103,12 +120,16 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
               make_map_bf16_3d(&mk, K, depth_kv, N, D, FWD_BN) &&
               make_map_bf16_3d(&mv, V, depth_kv, N, D, FWD_BN));
     if (!maps_ok) return FA_ERR_CUDA;
-    const int di = F8 ? 2 : (D == 128) ? 1 : 0;
-    if (!ds->fwd_attr[di]) {
-        if (cudaFuncSetAttribute(fa_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess)
-            return FA_ERR_CUDA;
-        ds->fwd_attr[di] = true;
+    const int di = F8 ? 2 : ((D == 128) ? 1 : 0) + (DROP ? 3 : 0);
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!ds->fwd_attr[di]) {
+            if (cudaFuncSetAttribute(fa_fwd_kernel<D, F8, DROP>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM_BYTES) != cudaSuccess)
+                return FA_ERR_CUDA;
+            ds->fwd_attr[di] = true;
+        }
     }
     FwdParams p;
     p.O = static_cast<__nv_bfloat16*>(O);
@@ -117,6 +138,11 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     p.n_kv_blocks = (N + FWD_BN - 1) / FWD_BN;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * scale_qk * 1.4426950408889634);
     p.o_scale = scale_v;
+    p.drop = DropoutParams{};
+    if (DROP) {
+        p.drop = *drop;
+        p.o_scale = scale_v * drop->keep_scale;
+    }
     p.causal = causal ? 1 : 0;
     p.err = ds->err;
     p.n_heads = B * H;
@@ -127,8 +153,18 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     const long long n_ctas = static_cast<long long>(p.n_pairs) * p.n_heads;
     if (n_ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
     dim3 grid(static_cast<unsigned>(n_ctas));
-    fa_fwd_kernel<D, F8><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+    fa_fwd_kernel<D, F8, DROP><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+bool ensure_bwd_attributes(DeviceState* ds, int d, bool drop) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    const int di = ((d == 128) ? 1 : 0) + (drop ? 2 : 0);
+    if (!ds->bwd_attr[di]) {
+        if (!bwd_set_attributes(d, drop)) return false;
+        ds->bwd_attr[di] = true;
+    }
+    return true;
 }
 
 // Self-test of the bounded-wait path: warp 0 waits, with a short limit, on a
@@ -162,6 +198,30 @@ fa_selftest_wait_kernel(uint32_t* err, unsigned long long timeout_ns, int* relea
 using namespace fa;
 
 extern "C" {
+
+fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                             const int* seqlens, int B, int H, int H_kv, int N, int d,
+                             float scale, int causal, float dropout_p, unsigned long long seed,
+                             unsigned int offset, cudaStream_t stream) {
+    DropoutParams drop;
+    bool on = false;
+    fa_status st = make_dropout(dropout_p, seed, offset, &drop, &on);
+    if (st != FA_OK) return st;
+    if (!on) return fa_forward_varlen(Q, K, V, O, LSE, seqlens, B, H, H_kv, N, d, scale, causal,
+                                      stream);
+    if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+        return FA_ERR_INVALID_ARG;
+    if ((st = check_shape(B, H, N, d, scale)) != FA_OK) return st;
+    if ((st = check_heads(H, H_kv)) != FA_OK) return st;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    return d == 128 ? launch_forward<128, false, true>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens,
+                                                       scale, causal, stream, 1.0, 1.f, &drop)
+                    : launch_forward<64, false, true>(ds, Q, K, V, O, LSE, B, H, H_kv, N, seqlens,
+                                                      scale, causal, stream, 1.0, 1.f, &drop);
+}
 
 fa_status fa_forward_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
                             const int* seqlens, int B, int H, int H_kv, int N, int d,
@@ -216,6 +276,34 @@ size_t fa_backward_workspace_bytes(int B, int H, int N, int d) {
     return bwd_workspace_bytes(B, H, N, d);
 }
 
+fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                              void* workspace, size_t workspace_bytes, const int* seqlens, int B,
+                              int H, int H_kv, int N, int d, float scale, int causal,
+                              float dropout_p, unsigned long long seed, unsigned int offset,
+                              cudaStream_t stream) {
+    DropoutParams drop;
+    bool on = false;
+    fa_status st = make_dropout(dropout_p, seed, offset, &drop, &on);
+    if (st != FA_OK) return st;
+    if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace)
+        return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
+    const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return FA_ERR_INVALID_ARG;
+    if ((st = check_shape(B, H, N, d, scale)) != FA_OK) return st;
+    if ((st = check_heads(H, H_kv)) != FA_OK) return st;
+    if (workspace_bytes < bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    if (!ensure_bwd_attributes(ds, d, on)) return FA_ERR_CUDA;
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, H_kv, N, d, seqlens,
+                      scale, causal, ds->err, on ? &drop : nullptr, stream)
+               ? FA_OK
+               : FA_ERR_CUDA;
+}
+
 fa_status fa_backward_varlen(const void* Q, const void* K, const void* V, const void* O,
                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                              void* workspace, size_t workspace_bytes, const int* seqlens, int B,
@@ -233,13 +321,9 @@ fa_status fa_backward_varlen(const void* Q, const void* K, const void* V, const 
     if (workspace_bytes < bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
     DeviceState* ds = current_device(&st);
     if (!ds) return st;
-    const int di = (d == 128) ? 1 : 0;
-    if (!ds->bwd_attr[di]) {
-        if (!bwd_set_attributes(d)) return FA_ERR_CUDA;
-        ds->bwd_attr[di] = true;
-    }
+    if (!ensure_bwd_attributes(ds, d, false)) return FA_ERR_CUDA;
     return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, H_kv, N, d, seqlens,
-                      scale, causal, ds->err, stream)
+                      scale, causal, ds->err, nullptr, stream)
                ? FA_OK
                : FA_ERR_CUDA;
 }
@@ -357,17 +441,13 @@ extern "C" fa_status fa_backward_noalloc(const void* Q, const void* K, const voi
             nd.ready = true;
         }
         scratch = nd.scratch;
-        const int di = (d == 128) ? 1 : 0;
-        if (!ds->bwd_attr[di]) {
-            if (!bwd_set_attributes(d)) return FA_ERR_CUDA;
-            ds->bwd_attr[di] = true;
-        }
     }
+    if (!ensure_bwd_attributes(ds, d, false)) return FA_ERR_CUDA;
     // Same three kernels as fa_backward; the preprocess kernel rewrites every
     // byte of the scratch the later kernels read (D, LSE and the zeroed fp32
     // dQ accumulator), so what an earlier call left there does not matter.
     return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, scratch, B, H, H, N, d, nullptr, scale,
-                      causal, ds->err, stream)
+                      causal, ds->err, nullptr, stream)
                ? FA_OK
                : FA_ERR_CUDA;
 }

@@ -28,6 +28,7 @@
 
 #include <algorithm>
 
+#include "philox.cuh"
 #include "sm100.cuh"
 #include "tma_host.h"
 
@@ -95,6 +96,7 @@ struct BwdParams {
     float scale, scale_log2;
     int causal;
     uint32_t* err;
+    DropoutParams drop;  // attention dropout (kernels instantiated with DROP only)
 };
 
 // ---------------------------------------------------------------------------
@@ -179,7 +181,12 @@ fa_bwd_dq_kernel(const float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dQ
 //   MMA:      S(0) dP(0) dV(0) | S(1) dK(0) dQ(0) dP(1) dV(1) | S(2) dK(1) ...
 // so the exp work of block i+1 overlaps the dK/dQ MMAs of block i.  With one
 // stage (d = 128: shared memory is full) the MMAs run in plain order.
-template <int D>
+// DROP: attention dropout (philox.cuh).  With Pd = P z / (1 - p) the forward
+// output is sum_j Pd_ij v_j, so dV takes Pd^T and dS takes the dropped dP:
+//     dV_j += sum_i Pd_ij dO_i,   dS_ij = P_ij (z_ij dP_ij / (1 - p) - D_i)
+// (D_i = <dO_i, O_i> is unchanged).  The keep bits are regenerated from the
+// same counters as the forward's.
+template <int D, bool DROP = false>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapdO,
@@ -392,6 +399,8 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         const uint32_t sDSrow = smem_u32(smem + C::OFF_DS + half * 16384) + r * 128;
         const uint32_t sDQ = smem_u32(smem + C::OFF_DQ);
         float pv[64];  // P^T (then dS^T) for this thread's 64 queries
+        uint32_t keep_lo = ~0u, keep_hi = ~0u;  // dropout keep bits of those queries
+        auto kept = [&](int c) { return (((c < 32) ? keep_lo : keep_hi) >> (c & 31)) & 1u; };
         bool ok = true;
 
         // ---- P(it): P^T = exp2(S^T * scale*log2e - LSE2[q])
@@ -400,6 +409,14 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             const uint32_t ph = (it / C::QS) & 1;
             const int q0 = q_block0(it);
             const int qh = q0 + 64 * half;  // first query of this warp's columns
+            if constexpr (DROP) {
+                // Made before S^T is ready: they depend only on the indices.
+                const unsigned long long M = keep_bits_key_row(
+                    p.drop, static_cast<uint32_t>(key), static_cast<uint32_t>(qh),
+                    static_cast<uint32_t>(q_head(it)), lane);
+                keep_lo = static_cast<uint32_t>(M);
+                keep_hi = static_cast<uint32_t>(M >> 32);
+            }
             if (!mbar_wait(&bars->q_full[s], ph, g, 29)) return false;
             if (!mbar_wait_warp(&bars->s_full, it & 1, g, 30)) return false;
             tc_fence_after();
@@ -441,8 +458,16 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             }
             {
                 uint32_t pk[32];
+                if constexpr (DROP) {
+                    const float ks = p.drop.keep_scale;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+                    for (int c = 0; c < 32; ++c)
+                        pk[c] = pack_bf16x2(kept(2 * c) ? pv[2 * c] * ks : 0.f,
+                                            kept(2 * c + 1) ? pv[2 * c + 1] * ks : 0.f);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pv[2 * c], pv[2 * c + 1]);
+                }
                 tmem_st32(tmem_addr(tmem, lane_base, C::T_PT + 32 * half), pk);
             }
             tmem_st_wait();
@@ -469,7 +494,9 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int c = 4 * c4 + e;
-                        pv[c] = pv[c] * (__uint_as_float(u[c]) - dv[e]);
+                        float dp = __uint_as_float(u[c]);
+                        if constexpr (DROP) dp = kept(c) ? dp * p.drop.keep_scale : 0.f;
+                        pv[c] = pv[c] * (dp - dv[e]);
                     }
                 }
             }
@@ -577,19 +604,23 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-inline bool bwd_set_attributes(int d) {
-    if (d == 64)
-        return cudaFuncSetAttribute(fa_bwd_main_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    BwdCfg<64>::SMEM_BYTES) == cudaSuccess;
-    return cudaFuncSetAttribute(fa_bwd_main_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                BwdCfg<128>::SMEM_BYTES) == cudaSuccess;
+template <int D, bool DROP>
+inline bool bwd_set_attributes_t() {
+    return cudaFuncSetAttribute(fa_bwd_main_kernel<D, DROP>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                BwdCfg<D>::SMEM_BYTES) == cudaSuccess;
 }
 
-template <int D>
+inline bool bwd_set_attributes(int d, bool drop) {
+    if (d == 64) return drop ? bwd_set_attributes_t<64, true>() : bwd_set_attributes_t<64, false>();
+    return drop ? bwd_set_attributes_t<128, true>() : bwd_set_attributes_t<128, false>();
+}
+
+template <int D, bool DROP>
 bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                   const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
                   int Hkv, int N, const int* seqlens, float scale, int causal, uint32_t* err,
-                  cudaStream_t stream) {
+                  const DropoutParams& drop, cudaStream_t stream) {
     const int Npad = static_cast<int>(round_up_128(N));
     const long long rows_pad = static_cast<long long>(B) * H * Npad;
     float* Dvec = static_cast<float*>(workspace);
@@ -627,9 +658,10 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
         p.causal = causal ? 1 : 0;
         p.err = err;
+        p.drop = drop;
         dim3 grid(Npad / 128, Hkv, B);
-        fa_bwd_main_kernel<D><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
-                                                                                   mdq, p);
+        fa_bwd_main_kernel<D, DROP><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mdo, mdq, p);
         if (cudaGetLastError() != cudaSuccess) return false;
     }
     {
@@ -642,14 +674,19 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
     return true;
 }
 
+// drop = null: no dropout.
 inline bool bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                        const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
                        int Hkv, int N, int d, const int* seqlens, float scale, int causal,
-                       uint32_t* err, cudaStream_t stream) {
-    return d == 128 ? bwd_launch_t<128>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N,
-                                        seqlens, scale, causal, err, stream)
-                    : bwd_launch_t<64>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N,
-                                       seqlens, scale, causal, err, stream);
+                       uint32_t* err, const DropoutParams* drop, cudaStream_t stream) {
+    const DropoutParams none{};
+    const DropoutParams& dp = drop ? *drop : none;
+#define FA_BWD_LAUNCH(DD, DR)                                                                    \
+    bwd_launch_t<DD, DR>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N, seqlens, scale, \
+                         causal, err, dp, stream)
+    if (d == 128) return drop ? FA_BWD_LAUNCH(128, true) : FA_BWD_LAUNCH(128, false);
+    return drop ? FA_BWD_LAUNCH(64, true) : FA_BWD_LAUNCH(64, false);
+#undef FA_BWD_LAUNCH
 }
 
 }  // namespace fa

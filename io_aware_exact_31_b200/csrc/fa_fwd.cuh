@@ -32,6 +32,7 @@
 // when the softmax warps may rescale O_t in place.
 #pragma once
 
+#include "philox.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -82,6 +83,7 @@ struct FwdParams {
     const int* seqlens; // [B] real tokens per batch (device), or null: all N are real
     int n_pairs;        // ceil(N / 256)
     uint32_t* err;      // device error word
+    DropoutParams drop; // attention dropout (kernels instantiated with DROP only)
 };
 
 // Barrier slots inside the barrier area.
@@ -92,10 +94,13 @@ struct FwdBars {
     uint64_t s_full[2], p_full[2][2], o_full[2];  // p_full[tile][key half]
 };
 
-template <int D, bool F8 = false>
+// DROP: attention dropout (philox.cuh) on the bf16 path; the 1 / (1 - p)
+// factor arrives folded into p.o_scale.
+template <int D, bool F8 = false, bool DROP = false>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
               const __grid_constant__ CUtensorMap mapV, const FwdParams p) {
+    static_assert(!(F8 && DROP), "dropout is implemented for bf16 operands only");
     using C = FwdCfg<D, F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -320,6 +325,24 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         const int nt = n_tile[t];
         const int tile_first_q = q0 + t * FWD_BM;
         for (int j = 0; j < nt; ++j) {
+            // Dropout keep bits of this row for keys [128 j, 128 j + 128):
+            // bit b of keep[w] for key 128 j + 32 w + b.  They depend only on
+            // the indices, so they are made while S_t(j) is still on the
+            // tensor core.
+            uint32_t keep[4] = {~0u, ~0u, ~0u, ~0u};
+            if constexpr (DROP) {
+                const uint32_t g0 = static_cast<uint32_t>(j * FWD_BN) >> 2;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) keep[w] = 0;
+#pragma unroll 1
+                for (int k = 0; k < 8; ++k) {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        keep[w] |= keep_nibble(p.drop, g0 + 8 * w + k, static_cast<uint32_t>(q),
+                                               static_cast<uint32_t>(bh))
+                                   << (4 * k);
+                }
+            }
             if (!(ok = mbar_wait_warp(&bars->s_full[t], j & 1, g, 9 + t))) break;
             tc_fence_after();
             uint32_t sr[128];
@@ -414,6 +437,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     } else {
                         pk[i] = pack_bf16x2(pe.x, pe.y);
                         ar[i % 4] = __fadd2_rn(ar[i % 4], unpack_bf16x2(pk[i]));
+                        if constexpr (DROP) {
+                            // Dropped weights leave the P.V product but stay in
+                            // both row sums (the softmax is of undropped scores).
+                            const uint32_t kb = keep[(h * 64 + 2 * i) / 32] >> ((2 * i) % 32);
+                            pk[i] &= ((kb & 1u) ? 0x0000FFFFu : 0u) | ((kb & 2u) ? 0xFFFF0000u : 0u);
+                        }
                     }
                 }
                 if constexpr (F8) tmem_st16(tS + h * C::P_COLS_HALF, pk);
