@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 METRIC = "fused attention fwd/bwd TFLOP/s and % of B200 dense-BF16 tensor-core peak"
 UNIT = "TFLOP/s"
 HEADLINE = "b4_h16_n4096_d128"
+DROPOUT_P = 0.1  # attention-dropout rate of the dropout extras (the pages' attn_dropout = 0.1)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -49,7 +50,7 @@ def load_peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha1()
-    for name in ("fa_fwd.cuh", "sm100.cuh"):
+    for name in ("fa_fwd.cuh", "sm100.cuh", "philox.cuh"):
         with open(os.path.join(ROOT, "io_aware_exact_31_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]
@@ -338,6 +339,27 @@ def run_gpu(args):
     del bq, q8, k8, v8, o8, l8
     torch.cuda.empty_cache()
 
+    # ---------------- extra: the headline forward with attention dropout p = 0.1
+    _, bd, _ = fwd_setup(w)
+    qd, kd, vd, od, ld = bd
+
+    def drop_fwd_step():
+        binding.forward(qd, kd, vd, causal=w.causal, scale=w.scale, out=od, lse=ld,
+                        dropout_p=DROPOUT_P, seed=1234, offset=0, stream=stream)
+
+    for _ in range(args.warmup):
+        drop_fwd_step()
+    msd = max_ranks(time_region(drop_fwd_step, args.steps, stream, barrier)) / args.steps
+    st, site = binding.check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {site:#x}")
+    extra[w.name + "_dropout"] = {"pass": "fwd", "dropout_p": DROPOUT_P, "ms": round(msd, 4),
+                                  "tflops": round(w.fwd_flops / (msd * 1e-3) / 1e12, 1),
+                                  "frac_of_bf16_peak": round(w.fwd_flops / (msd * 1e-3) / 1e12 /
+                                                             peaks["bf16_tflops"], 4)}
+    del bd, qd, kd, vd, od, ld
+    torch.cuda.empty_cache()
+
     # ---------------- extra: forward + backward workload
     w5 = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
     x5 = workload_inputs(w5, seed=rank)
@@ -354,18 +376,35 @@ def run_gpu(args):
     def fwd5_step():
         binding.forward(q5, k5, v5, causal=True, scale=w5.scale, out=o5, lse=l5)
 
+    def bwd5_drop_step():
+        binding.backward(q5, k5, v5, o5, do5, l5, causal=True, scale=w5.scale, dq=dq5, dk=dk5,
+                         dv=dv5, workspace=ws, dropout_p=DROPOUT_P, seed=99, offset=0)
+
+    def fwd5_drop_step():
+        binding.forward(q5, k5, v5, causal=True, scale=w5.scale, out=o5, lse=l5,
+                        dropout_p=DROPOUT_P, seed=99, offset=0)
+
     for _ in range(args.warmup):
         bwd_step()
         fwd5_step()
     msb = max_ranks(time_region(bwd_step, args.steps, stream, barrier)) / args.steps
     msf = max_ranks(time_region(fwd5_step, args.steps, stream, barrier)) / args.steps
+    for _ in range(args.warmup):
+        fwd5_drop_step()
+        bwd5_drop_step()
+    msfd = max_ranks(time_region(fwd5_drop_step, args.steps, stream, barrier)) / args.steps
+    msbd = max_ranks(time_region(bwd5_drop_step, args.steps, stream, barrier)) / args.steps
     st, site = binding.check_device_error()
     if st != 0:
         raise RuntimeError(f"device error {site:#x}")
     extra[w5.name] = {"pass": "fwd+bwd", "fwd_ms": round(msf, 4), "bwd_ms": round(msb, 4),
                       "fwd_tflops": round(w5.fwd_flops / (msf * 1e-3) / 1e12, 1),
                       "bwd_tflops": round(w5.bwd_flops / (msb * 1e-3) / 1e12, 1),
-                      "bwd_launches_per_step": 3}
+                      "bwd_launches_per_step": 3,
+                      "dropout": {"p": DROPOUT_P, "fwd_ms": round(msfd, 4),
+                                  "bwd_ms": round(msbd, 4),
+                                  "fwd_tflops": round(w5.fwd_flops / (msfd * 1e-3) / 1e12, 1),
+                                  "bwd_tflops": round(w5.bwd_flops / (msbd * 1e-3) / 1e12, 1)}}
 
     traffic = recorded_traffic()
     achieved = per_gpu

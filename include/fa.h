@@ -92,18 +92,21 @@ fa_status fa_forward_varlen(const void *Q, const void *K, const void *V, void *O
  * Attention dropout (the attn_dropout option of downcodes.com "triton
  * transformer", usage section; the page gives no formula).  Inverted dropout
  * on the normalised probabilities:
- *     O_i = sum_j P_ij z_ij / (1 - dropout_p) v_j,   LSE as without dropout
+ *     O_i = sum_j P_ij z_ij / q v_j,   LSE as without dropout
  * with the keep bit z_ij of query i, key j of query head bh = b * H + h taken
  * from the counter-based generator Philox-4x32-10 (Salmon et al., "Parallel
  * Random Numbers: As Easy as 1, 2, 3", SC'11):
- *     w = Philox(counter = (j / 4, i, bh, offset), key = (seed & 0xffffffff, seed >> 32))
- *     z_ij = (w[j % 4] < floor((1 - dropout_p) * 2^32))
- * (i, j counted from the start of the sequence).  The same (seed, offset)
- * given to fa_backward_dropout regenerates the mask; a caller that needs a
- * fresh mask per call changes either.
- *   dropout_p : in [0, 1) (FA_ERR_INVALID_ARG otherwise, NaN included);
- *               0 -- or any value with floor((1 - p) 2^32) = 2^32 -- is
- *               exactly fa_forward_varlen.
+ *     W = Philox(counter = (j / 8, i, bh, offset), key = (seed & 0xffffffff, seed >> 32))
+ *     u = (W[(j % 8) / 2] >> (16 * (j % 2))) & 0x7fff        (15-bit uniform)
+ *     z_ij = (u < t),  t = floor((1 - dropout_p) * 2^15 + 1/2),  q = t / 2^15
+ * (i, j counted from the start of the sequence).  q, the keep probability, is
+ * the multiple of 2^-15 nearest to 1 - dropout_p, and dividing by it keeps
+ * the output unbiased.  The same (seed, offset) given to fa_backward_dropout
+ * regenerates the mask; a caller that needs a fresh mask per call changes
+ * either.
+ *   dropout_p : in [0, 1 - 2^-16] (FA_ERR_INVALID_ARG otherwise, NaN
+ *               included); values below 2^-16 (t = 2^15) are exactly
+ *               fa_forward_varlen.
  * Other arguments as fa_forward_varlen (seqlens may be NULL; K/V with H_kv
  * heads).  The keep-bit generation costs integer work in the softmax warps.
  */
@@ -181,8 +184,8 @@ fa_status fa_backward_varlen(const void *Q, const void *K, const void *V, const 
 /*
  * Backward of fa_forward_dropout: the same (dropout_p, seed, offset) and
  * seqlens as the forward call that produced O and LSE.  With
- * Pd_ij = P_ij z_ij / (1 - p):  dV_j = sum_i Pd_ij dO_i,
- * dS_ij = P_ij (z_ij <dO_i, v_j> / (1 - p) - <dO_i, O_i>), dQ and dK from dS
+ * Pd_ij = P_ij z_ij / q:  dV_j = sum_i Pd_ij dO_i,
+ * dS_ij = P_ij (z_ij <dO_i, v_j> / q - <dO_i, O_i>), dQ and dK from dS
  * as in fa_backward.  Other arguments as fa_backward_varlen.
  */
 fa_status fa_backward_dropout(const void *Q, const void *K, const void *V, const void *O,

@@ -85,18 +85,26 @@ fa_status check_heads(int H, int Hkv) {
     return FA_OK;
 }
 
-// Attention-dropout parameters from (p, seed, offset).  *on = false when p
-// is so small that 1 - p rounds to 1 (floor((1 - p) 2^32) = 2^32: nothing is
-// ever dropped), which runs the kernels without dropout.
+// Attention-dropout parameters from (p, seed, offset): keep threshold
+// t = floor((1 - p) 2^15 + 1/2) on 15-bit uniforms, keep scale 2^15 / t, and
+// the ten Philox round keys.  *on = false when t = 2^15 (p < 2^-16: nothing is
+// ever dropped), which runs the kernels without dropout; t = 0 is rejected.
 fa_status make_dropout(float p, uint64_t seed, uint32_t offset, DropoutParams* d, bool* on) {
     if (!(p >= 0.f && p < 1.f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
-    const double t = std::floor((1.0 - static_cast<double>(p)) * 4294967296.0);
-    *on = t < 4294967296.0;
-    d->seed_lo = static_cast<uint32_t>(seed);
-    d->seed_hi = static_cast<uint32_t>(seed >> 32);
+    const double t = std::floor((1.0 - static_cast<double>(p)) * 32768.0 + 0.5);
+    if (t < 1.0) return FA_ERR_INVALID_ARG;
+    *on = t < 32768.0;
+    uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        d->key[2 * r] = k0;
+        d->key[2 * r + 1] = k1;
+        k0 += 0x9E3779B9u;  // Weyl increments of Philox-4x32
+        k1 += 0xBB67AE85u;
+    }
     d->offset = offset;
-    d->threshold = *on ? static_cast<uint32_t>(t) : 0xFFFFFFFFu;
-    d->keep_scale = static_cast<float>(1.0 / (1.0 - static_cast<double>(p)));
+    const uint32_t ref = (static_cast<uint32_t>(t) - 1u) | 0x8000u;
+    d->lanes_ref = ref | (ref << 16);
+    d->keep_scale = static_cast<float>(32768.0 / t);
     return FA_OK;
 }
 

@@ -325,24 +325,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         const int nt = n_tile[t];
         const int tile_first_q = q0 + t * FWD_BM;
         for (int j = 0; j < nt; ++j) {
-            // Dropout keep bits of this row for keys [128 j, 128 j + 128):
-            // bit b of keep[w] for key 128 j + 32 w + b.  They depend only on
-            // the indices, so they are made while S_t(j) is still on the
-            // tensor core.
+            // Dropout keep bits of this row for keys [128 j, 128 j + 128)
+            // (layout of keep_bits_row128).  They depend only on the indices,
+            // so they are made while S_t(j) is still on the tensor core.
             uint32_t keep[4] = {~0u, ~0u, ~0u, ~0u};
-            if constexpr (DROP) {
-                const uint32_t g0 = static_cast<uint32_t>(j * FWD_BN) >> 2;
-#pragma unroll
-                for (int w = 0; w < 4; ++w) keep[w] = 0;
-#pragma unroll 1
-                for (int k = 0; k < 8; ++k) {
-#pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        keep[w] |= keep_nibble(p.drop, g0 + 8 * w + k, static_cast<uint32_t>(q),
-                                               static_cast<uint32_t>(bh))
-                                   << (4 * k);
-                }
-            }
+            if constexpr (DROP)
+                keep_bits_row128(p.drop, static_cast<uint32_t>(j * FWD_BN), static_cast<uint32_t>(q),
+                                 static_cast<uint32_t>(bh), keep);
             if (!(ok = mbar_wait_warp(&bars->s_full[t], j & 1, g, 9 + t))) break;
             tc_fence_after();
             uint32_t sr[128];
@@ -440,8 +429,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                         if constexpr (DROP) {
                             // Dropped weights leave the P.V product but stay in
                             // both row sums (the softmax is of undropped scores).
-                            const uint32_t kb = keep[(h * 64 + 2 * i) / 32] >> ((2 * i) % 32);
-                            pk[i] &= ((kb & 1u) ? 0x0000FFFFu : 0u) | ((kb & 2u) ? 0xFFFF0000u : 0u);
+                            // keys 64h + 2i (low half) and 64h + 2i + 1 (high half)
+                            const int o = (2 * i) % 32;
+                            const uint32_t kb =
+                                (keep[(h * 64 + 2 * i) / 32] >> (4 * (o / 8) + (o % 8) / 2)) & 0x00010001u;
+                            pk[i] &= kb * 0xFFFFu;
                         }
                     }
                 }

@@ -57,11 +57,18 @@
  *           z_ij comes from the counter-based generator Philox-4x32-10
  *           (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as
  *           1, 2, 3", SC'11), called with
- *             counter = (j / 4, i, b * H + h, offset), key = (seed mod 2^32,
+ *             counter = (j / 8, i, b * H + h, offset), key = (seed mod 2^32,
  *                       seed / 2^32)
- *           and z_ij = 1 iff word (j mod 4) of the output is below
- *           floor((1 - p) 2^32), for query i, key j of query head h of
- *           batch b (positions counted from the start of the sequence).
+ *           for query i, key j of query head h of batch b (positions counted
+ *           from the start of the sequence).  Each 32-bit output word holds
+ *           two 15-bit numbers, u = (word >> 16 e) mod 2^15 for e = 0, 1;
+ *           key j takes word (j mod 8) / 2, half e = j mod 2, and is kept iff
+ *           u < t = floor((1 - p) 2^15 + 1/2).  The keep probability is then
+ *           q = t / 2^15 (the nearest multiple of 2^-15 to 1 - p) and kept
+ *           weights are scaled by 1 / q, so the dropout stays unbiased:
+ *             O_i = sum_j P_ij z_ij / q v_j.
+ *           t = 2^15 (p < 2^-16) keeps everything; p > 1 - 2^-16 (t = 0)
+ *           is rejected.
  *
  * Every function returns 0 on success, -1 on a bad argument, -2 if memory
  * could not be allocated.
@@ -142,33 +149,37 @@ void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t
 
 /* [DROP] parameters; NULL or p == 0 means no dropout. */
 struct dropout {
-    double p;            /* probability of dropping, [0, 1) */
+    double p;            /* requested probability of dropping, [0, 1) */
     uint32_t key[2];     /* the seed */
     uint32_t offset;     /* counter word 3 */
-    uint64_t threshold;  /* floor((1 - p) 2^32): keep iff word < threshold */
-    double keep_scale;   /* 1 / (1 - p) */
+    uint32_t threshold;  /* t = floor((1 - p) 2^15 + 1/2): keep iff u < t */
+    double keep_scale;   /* 2^15 / t = 1 / (keep probability) */
 };
 
 static int make_dropout(struct dropout *dr, double p, uint64_t seed, uint32_t offset)
 {
     if (!(p >= 0.0 && p < 1.0))
         return -1;
+    const double t = floor((1.0 - p) * 32768.0 + 0.5);
+    if (t < 1.0)
+        return -1;
     dr->p = p;
     dr->key[0] = (uint32_t)seed;
     dr->key[1] = (uint32_t)(seed >> 32);
     dr->offset = offset;
-    dr->threshold = (uint64_t)floor((1.0 - p) * 4294967296.0);
-    dr->keep_scale = 1.0 / (1.0 - p);
+    dr->threshold = (uint32_t)t;
+    dr->keep_scale = 32768.0 / t;
     return 0;
 }
 
 /* z_ij of [DROP] for query i, key j of query head bh = b * H + h. */
 static int dropout_keep(const struct dropout *dr, int64_t bh, int64_t i, int64_t j)
 {
-    const uint32_t ctr[4] = {(uint32_t)(j / 4), (uint32_t)i, (uint32_t)bh, dr->offset};
+    const uint32_t ctr[4] = {(uint32_t)(j / 8), (uint32_t)i, (uint32_t)bh, dr->offset};
     uint32_t w[4];
     oracle_philox4x32_10(ctr, dr->key, w);
-    return (uint64_t)w[j % 4] < dr->threshold;
+    const uint32_t u = (w[(j % 8) / 2] >> (16 * (j % 2))) & 0x7FFFu;
+    return u < dr->threshold;
 }
 
 /* The [DROP] keep mask z as bytes [B, H, N, N] (row = query, column = key). */
@@ -366,9 +377,9 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
  * of these over the query heads that share it.  With [PAD] lengths each
  * (batch, head) is the same on its first len tokens (P = 0 outside) and all
  * gradients of padding tokens are 0.  With [DROP] the output is
- * O_i = sum_j Pd_ij v_j, Pd_ij = P_ij z_ij / (1 - p), and by the chain rule
+ * O_i = sum_j Pd_ij v_j, Pd_ij = P_ij z_ij / q, and by the chain rule
  *   dV_j  = sum_i Pd_ij dO_i
- *   dP_ij = <dO_i, v_j> z_ij / (1 - p)       (gradient with respect to P)
+ *   dP_ij = <dO_i, v_j> z_ij / q             (gradient with respect to P)
  * with D, dS, dQ, dK as above (D_i = sum_j P_ij dP_ij still equals
  * <dO_i, O_i>).  dQ is double [B,H,N,d]; dK, dV are double [B,Hkv,N,d].
  */
@@ -386,7 +397,7 @@ int oracle_attention_backward_dropout(const void *Q, const void *K, const void *
     const struct dropout *dr = p_drop > 0.0 ? &drop : NULL;
     double *P = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
     double *dS = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
-    /* z_ij / (1 - p) of the current head (only with dropout) */
+    /* z_ij / q of the current head (only with dropout) */
     double *Z = dr ? (double *)malloc((size_t)N * (size_t)N * sizeof(double)) : NULL;
     if (!P || !dS || (dr && !Z)) {
         free(P);

@@ -4,7 +4,8 @@ against the fp64 oracle with the same Philox-4x32-10 keep mask.
 
 Two kinds of check:
   * mask read-back, bit-exact: with Q = 0 every score is 0, so every weight
-    is exactly 1 and O_i = sum_j z_ij v_j / (n_i (1 - p)) (n_i visible keys).
+    is exactly 1 and O_i = sum_j z_ij v_j / (n_i q) (n_i visible keys, q the
+    keep probability).
     A one-hot V (column c <- key c of one chunk) makes O[i, c] non-zero
     exactly where z_ij = 1.  Likewise a one-hot dO exposes z through dV in the
     backward (which regenerates the mask on its own).
@@ -69,10 +70,12 @@ def test_forward_mask_readback(B, H, Hkv, N, p, seqlens, causal, d):
     want = oracle.dropout_keep_mask(B, H, N, p, seed, offset) & vis
     mism = np.argwhere(got != want)
     assert mism.size == 0, f"{len(mism)} keep bits differ, first (b,h,i,j) = {mism[:5].tolist()}"
-    # kept weights are 1 / (n_i (1 - p)) up to the bf16 rounding of O
+    # kept weights are 1 / (n_i q) up to the bf16 rounding of O, with the keep
+    # probability q = t / 2^15, t = floor((1 - p) 2^15 + 1/2)
     n_i = vis.sum(-1)  # [B,1,N]
     vals = np.concatenate(o_kept, axis=-1)[..., :N]
-    expect = np.where(want, 1.0 / (np.maximum(n_i, 1)[..., None] * (1.0 - p)), 0.0)
+    q_keep = math.floor((1.0 - p) * 2.0 ** 15 + 0.5) / 2.0 ** 15
+    expect = np.where(want, 1.0 / (np.maximum(n_i, 1)[..., None] * q_keep), 0.0)
     assert np.allclose(vals, expect, rtol=2 ** -8, atol=0)
 
 
@@ -151,6 +154,9 @@ def test_dropout_zero_is_the_plain_path_and_masks_are_reproducible():
                                 99, 0, binding._stream_handle(None))
     assert st == binding.FA_OK
     assert torch.equal(o0, o1) and torch.equal(o0, o2) and torch.equal(l0, l2)
+    # p below 2^-16 rounds to keep probability 1: the plain path as well
+    o3, l3 = binding.forward(q, k, v, causal=True, dropout_p=1e-6, seed=99)
+    assert torch.equal(o0, o3) and torch.equal(l0, l3)
     a, la = binding.forward(q, k, v, causal=True, dropout_p=0.2, seed=5, offset=1)
     b, lb = binding.forward(q, k, v, causal=True, dropout_p=0.2, seed=5, offset=1)
     c, _ = binding.forward(q, k, v, causal=True, dropout_p=0.2, seed=5, offset=2)
@@ -160,7 +166,7 @@ def test_dropout_zero_is_the_plain_path_and_masks_are_reproducible():
 
 def test_dropout_rejects_bad_probability():
     z = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
-    for p in (1.0, -0.1, float("nan"), 1.5):
+    for p in (1.0, -0.1, float("nan"), 1.5, 1.0 - 2.0 ** -17):
         with pytest.raises(binding.FaError) as e:
             binding.forward(z, z, z, dropout_p=p, seed=1)
         assert e.value.status == binding.FA_ERR_INVALID_ARG

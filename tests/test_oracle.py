@@ -498,30 +498,43 @@ def pin_philox_known_answers(lib):
         assert tuple(int(x) for x in oracle.philox4x32_10(ctr, key, lib=lib)) == want
 
 
+def _keep_threshold(p):
+    """t = floor((1 - p) 2^15 + 1/2): keys are kept with probability t / 2^15."""
+    return math.floor((1.0 - p) * 2.0 ** 15 + 0.5)
+
+
 def pin_dropout_mask_convention(lib):
-    """Keep mask = the stated counter layout (j/4, i, b*H+h, offset), key =
-    seed halves, word j%4 below floor((1-p) 2^32), evaluated independently."""
+    """Keep mask = the stated counter layout (j/8, i, b*H+h, offset), key =
+    seed halves, 15-bit half (j%2) of word (j%8)/2 below t, evaluated
+    independently."""
     assert _philox_py(*PHILOX_KAT[2][:2]) == PHILOX_KAT[2][2]
-    B, H, N, p, seed, offset = 2, 3, 11, 0.3, 0x0123456789ABCDEF, 7
+    B, H, N, p, seed, offset = 2, 3, 19, 0.3, 0x0123456789ABCDEF, 7
     m = oracle.dropout_keep_mask(B, H, N, p, seed, offset, lib=lib)
-    t = math.floor((1.0 - p) * 2.0 ** 32)
+    t = _keep_threshold(p)
     key = (seed & 0xFFFFFFFF, seed >> 32)
     for b in range(B):
         for h in range(H):
             for i in range(N):
                 for j in range(N):
-                    w = _philox_py((j // 4, i, b * H + h, offset), key)[j % 4]
-                    assert m[b, h, i, j] == (w < t), (b, h, i, j)
+                    w = _philox_py((j // 8, i, b * H + h, offset), key)[(j % 8) // 2]
+                    u = (w >> (16 * (j % 2))) & 0x7FFF
+                    assert m[b, h, i, j] == (u < t), (b, h, i, j)
 
 
 def pin_dropout_keep_rate(lib):
-    """Each element is kept with probability 1 - p: the kept fraction of 2^20
-    draws is within 6 standard deviations; p = 0 keeps everything."""
-    for p in (0.1, 0.5, 0.9):
+    """Each element is kept with probability t / 2^15 (within 2^-16 of 1 - p):
+    the kept fraction of 2^20 draws is within 6 standard deviations; p = 0
+    and p < 2^-16 keep everything; p too close to 1 (t = 0) is rejected."""
+    for p in (0.1, 0.5, 0.9, 0.123456):
+        q = _keep_threshold(p) / 2.0 ** 15
+        assert abs(q - (1 - p)) <= 2.0 ** -16
         m = oracle.dropout_keep_mask(1, 4, 512, p, 99, 3, lib=lib)
         n = m.size
-        assert abs(m.mean() - (1 - p)) <= 6 * math.sqrt(p * (1 - p) / n), (p, m.mean())
+        assert abs(m.mean() - q) <= 6 * math.sqrt(q * (1 - q) / n), (p, m.mean())
     assert oracle.dropout_keep_mask(1, 1, 64, 0.0, 5, lib=lib).all()
+    assert oracle.dropout_keep_mask(1, 1, 64, 1e-6, 5, lib=lib).all()
+    with pytest.raises(RuntimeError):
+        oracle.dropout_keep_mask(1, 1, 8, 1.0 - 2.0 ** -17, 5, lib=lib)
 
 
 def pin_dropout_zero_is_plain_attention(lib):
@@ -533,7 +546,8 @@ def pin_dropout_zero_is_plain_attention(lib):
 
 
 def _dropout_torch(Q, K, V, z, p, scale, causal, seqlens):
-    """(softmax(scale Q K^T, masked) * z / (1 - p)) V in fp64 torch, with grads."""
+    """(softmax(scale Q K^T, masked) * z / q) V in fp64 torch, with grads
+    (q = t / 2^15, the keep probability)."""
     B, H, N, _ = Q.shape
     G = H // K.shape[1]
     tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
@@ -541,7 +555,8 @@ def _dropout_torch(Q, K, V, z, p, scale, causal, seqlens):
     s = (scale * tq @ tk.repeat_interleave(G, dim=1).transpose(-1, -2)).masked_fill(
         ~mask, float("-inf"))
     P = torch.softmax(s, dim=-1)
-    out = (P * torch.from_numpy(z.astype(np.float64)) / (1.0 - p)) @ tv.repeat_interleave(G, dim=1)
+    q = _keep_threshold(p) / 2.0 ** 15
+    out = (P * torch.from_numpy(z.astype(np.float64)) / q) @ tv.repeat_interleave(G, dim=1)
     return out, torch.logsumexp(s, dim=-1), (tq, tk, tv)
 
 
@@ -675,10 +690,12 @@ MUTANTS = {
     "merge_max_wrong": ("const double mm = fmax(m_x, m_y);", "const double mm = m_x;", 0),
     "philox_seven_rounds": ("for (int r = 0; r < 10; ++r) {", "for (int r = 0; r < 7; ++r) {", 0),
     "philox_hi_lo_swapped": ("c1 = (uint32_t)p1;", "c1 = (uint32_t)(p1 >> 32);", 0),
-    "drop_counter_transposed": ("{(uint32_t)(j / 4), (uint32_t)i,", "{(uint32_t)(i / 4), (uint32_t)j,", 0),
-    "drop_word_index": ("return (uint64_t)w[j % 4] <", "return (uint64_t)w[i % 4] <", 0),
-    "drop_keep_inverted": ("return (uint64_t)w[j % 4] < dr->threshold;",
-                           "return (uint64_t)w[j % 4] >= dr->threshold;", 0),
+    "drop_counter_transposed": ("{(uint32_t)(j / 8), (uint32_t)i,", "{(uint32_t)(i / 8), (uint32_t)j,", 0),
+    "drop_word_index": ("w[(j % 8) / 2]", "w[(i % 8) / 2]", 0),
+    "drop_half_index": (">> (16 * (j % 2))", ">> (16 * (i % 2))", 0),
+    "drop_16_bit_uniform": (") & 0x7FFFu;", ") & 0xFFFFu;", 0),
+    "drop_keep_inverted": ("return u < dr->threshold;", "return u >= dr->threshold;", 0),
+    "drop_scale_one_minus_p": ("dr->keep_scale = 32768.0 / t;", "dr->keep_scale = 1.0 / (1.0 - p);", 0),
     "drop_seed_halves_swapped": ("dr->key[0] = (uint32_t)seed;", "dr->key[0] = (uint32_t)(seed >> 32);", 0),
     "drop_no_keep_scale": ("? p * dr->keep_scale : 0.0;", "? p : 0.0;", 0),
     "drop_fwd_kv_head": ("scale, causal, dr, bh, s,", "scale, causal, dr, kv_head(bh, H, Hkv), s,", 0),
