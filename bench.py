@@ -212,6 +212,8 @@ def run_gpu(args):
     stream = torch.cuda.current_stream()
     sh = stream.cuda_stream
 
+    w = WORKLOADS[HEADLINE]
+
     def fwd_setup(w):
         x = workload_inputs(w, seed=rank)
         q, k, v = (x[n].cuda() for n in ("Q", "K", "V"))
@@ -226,11 +228,20 @@ def run_gpu(args):
         if st != 0:
             raise binding.FaError(st, "fa_forward")
 
+    if args.only == "fwd" and args.dropout > 0:
+        # profiler runs of the dropout forward: same workload, fa_forward_dropout
+        def launch_fwd(a):  # noqa: F811
+            st = lib.fa_forward_dropout(*a[:5], None, w.B, w.H, w.H, w.N, w.d, w.scale,
+                                        int(w.causal), args.dropout, 1234, 0,
+                                        binding.ctypes.c_void_p(a[-1]))
+            if st != 0:
+                raise binding.FaError(st, "fa_forward_dropout")
+
     if args.only == "bwd":
         return run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank), rank
 
     # ---------------- headline: forward on the 4x16x4096x128 workload
-    w = WORKLOADS[HEADLINE]
+
     x, bufs, fargs = fwd_setup(w)
     for _ in range(args.warmup):
         launch_fwd(fargs)
@@ -265,7 +276,7 @@ def run_gpu(args):
             dist.destroy_process_group()
         return {"metric": METRIC, "value": round(tflops, 1), "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-                "config": {"workload": f"{HEADLINE} fwd"}, "clocks": clocks,
+                "config": {"workload": f"{HEADLINE} fwd", "dropout_p": args.dropout}, "clocks": clocks,
                 "gpu_launches": args.steps}, rank
 
     # ---------------- e2e through the C ABI with host buffers
@@ -449,9 +460,13 @@ def run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank):
                      dtype=torch.uint8)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
 
+    p = args.dropout
+    if p > 0:
+        o, lse = binding.forward(q, k, v, causal=True, scale=w5.scale, dropout_p=p, seed=99)
+
     def step():
         binding.backward(q, k, v, o, do, lse, causal=True, scale=w5.scale, dq=dq, dk=dk, dv=dv,
-                         workspace=ws)
+                         workspace=ws, dropout_p=p, seed=99)
 
     for _ in range(args.warmup):
         step()
@@ -459,7 +474,8 @@ def run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank):
     ms = time_region(step, args.steps, stream, torch.cuda.synchronize) / args.steps
     return {"metric": METRIC, "value": round(w5.bwd_flops / (ms * 1e-3) / 1e12, 1),
             "unit": UNIT, "ms_per_step": round(ms, 4), "steps": args.steps,
-            "config": {"workload": f"{w5.name} bwd"}, "gpu_launches": 3 * args.steps}
+            "config": {"workload": f"{w5.name} bwd", "dropout_p": p},
+            "gpu_launches": 3 * args.steps}
 
 
 def oracle_sample(target_s: float, step_rows: int | None = None):
@@ -532,6 +548,8 @@ def main():
                     help="host time of one oracle step in --impl reference")
     ap.add_argument("--only", default=None, choices=[None, "fwd", "bwd"],
                     help="time only the headline forward / the backward (profiler runs)")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="attention-dropout rate of the --only fwd / --only bwd runs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target host time of the oracle CPU-baseline sample")
     args = ap.parse_args()
