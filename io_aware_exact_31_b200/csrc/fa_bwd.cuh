@@ -92,6 +92,7 @@ struct BwdParams {
     __nv_bfloat16* dV;
     int N, Npad, n_q_blocks;
     int H, group;        // query heads per batch; query heads per K/V head
+    int Hkv, n_kv_heads; // K/V heads per batch; B * Hkv
     const int* seqlens;  // [B] real tokens per batch (device), or null
     float scale, scale_log2;
     int causal;
@@ -203,13 +204,24 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     const uint32_t warp = warp_id(), lane = lane_id();
     // CTA = (key block, K/V head).  With grouped-query attention the CTA walks
     // every query head of its group, so dK/dV sum over the group in TMEM.
-    const int bkv = blockIdx.z * gridDim.y + blockIdx.y;  // K/V head (b * H_kv + h_kv)
-    const int bq0 = blockIdx.z * p.H + blockIdx.y * p.group;  // first query head of the group
-    const int kb = blockIdx.x;  // key block; causal: block 0 has the most work and starts first
+    // 1-D grid.  Causal: key-block-major, block 0 (the most query blocks) of
+    // every head first, so the heaviest CTAs never form the tail.
+    // Non-causal (equal work): head-major, the key blocks of one head
+    // adjacent, so the CTAs resident at one time stream few heads' Q and dO.
+    int kb, bkv;
+    if (p.causal) {
+        kb = static_cast<int>(blockIdx.x) / p.n_kv_heads;
+        bkv = static_cast<int>(blockIdx.x) % p.n_kv_heads;
+    } else {
+        bkv = static_cast<int>(blockIdx.x) / p.n_q_blocks;
+        kb = static_cast<int>(blockIdx.x) % p.n_q_blocks;
+    }
+    const int batch = bkv / p.Hkv;
+    const int bq0 = batch * p.H + (bkv % p.Hkv) * p.group;  // first query head of the group
     const int k0 = kb * BWD_BN;
     // Padded batches: only the first len tokens are real; a key block past len
     // has zero gradients, query blocks past len contribute nothing.
-    const int len = p.seqlens ? min(max(__ldg(p.seqlens + blockIdx.z), 0), p.N) : p.N;
+    const int len = p.seqlens ? min(max(__ldg(p.seqlens + batch), 0), p.N) : p.N;
     const bool padding_cta = k0 >= len;
     const int i_begin = p.causal ? kb : 0;  // first query block that sees this key block
     const int nq = padding_cta ? 0 : (len + BWD_BM - 1) / BWD_BM - i_begin;  // per query head
@@ -653,13 +665,17 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         p.n_q_blocks = Npad / 128;
         p.H = H;
         p.group = H / Hkv;
+        p.Hkv = Hkv;
+        p.n_kv_heads = B * Hkv;
         p.seqlens = seqlens;
         p.scale = scale;
         p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
         p.causal = causal ? 1 : 0;
         p.err = err;
         p.drop = drop;
-        dim3 grid(Npad / 128, Hkv, B);
+        const long long n_ctas = static_cast<long long>(Npad / 128) * B * Hkv;
+        if (n_ctas > 0x7fffffffLL) return false;
+        dim3 grid(static_cast<unsigned>(n_ctas));
         fa_bwd_main_kernel<D, DROP><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(
             mq, mk, mv, mdo, mdq, p);
         if (cudaGetLastError() != cudaSuccess) return false;
