@@ -23,7 +23,11 @@
 // dQ_i goes to 128-B-swizzled shared memory and is added to the fp32
 // accumulator with TMA tensor reduce-adds (one per 32-column box).
 // Warps: 0-7 compute (warp w: TMEM lane quarter w%4, column half w/4),
-// 8 MMA issuer (TMEM owner), 9 TMA producer, 10 dQ reducer, 11 idle.
+// 8 MMA issuer of S^T, dP^T and dV (TMEM owner), 9 TMA producer, 10 dQ
+// reducer, 11 MMA issuer of dK and dQ.  One thread issues a tcgen05.mma only
+// about every 110 clocks whatever its size, and at d = 64 three of the five
+// products have N = 64, so a single issuer would leave the tensor core idle
+// most of the time; two issuers share the 5 products 16 : 16 instructions.
 #pragma once
 
 #include <algorithm>
@@ -68,7 +72,6 @@ struct BwdCfg {
     // TMEM columns
     static constexpr uint32_t T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 256 + D;
     static constexpr bool DQ_ALIAS = (D == 128);  // dQ shares the dP^T columns
-    static constexpr bool EARLY_S = (QS >= 2);    // issue S^T(i+1) before dK/dQ(i)
     static constexpr uint32_t T_DQ = DQ_ALIAS ? T_DPT : 256 + 2 * D;
     // P^T: its own 64 columns when they exist (d = 64); over S^T otherwise,
     // which needs both column halves of a lane read before either writes.
@@ -177,14 +180,14 @@ fa_bwd_dq_kernel(const float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dQ
 //   P(i):   P^T = exp2(S^T * scale*log2e - LSE2[q])  (TMEM -> regs -> TMEM)
 //   dS(i):  dS^T = P^T * (dP^T - D[q])               (-> swizzled smem, bf16)
 //   dQr(i): dQ_i from TMEM -> swizzled fp32 smem staging for the reducer warp
-// With two Q/dO stages (d = 64) the work is software-pipelined:
+// and the work is software-pipelined across the two MMA issuers:
 //   compute:  P(0) dS(0) | P(1) dQr(0) dS(1) | P(2) dQr(1) dS(2) | ... dQr(n-1)
-//   MMA:      S(0) dP(0) dV(0) | S(1) dK(0) dQ(0) dP(1) dV(1) | S(2) dK(1) ...
-// so the exp work of block i+1 overlaps the dK/dQ MMAs of block i.  With one
-// stage (d = 128: shared memory is full) the MMAs run in plain order.
-// DROP: attention dropout (philox.cuh).  With Pd = P z / (1 - p) the forward
+//   MMA 8:    S(0) dP(0) dV(0) S(1) dP(1) dV(1) S(2) ...   (dP(i+1) after dS(i) is read)
+//   MMA 11:   dK(0) dQ(0) dK(1) dQ(1) ...                   (each after dS(i) is stored)
+// so the exp work of block i+1 overlaps the dK/dQ MMAs of block i.
+// DROP: attention dropout (philox.cuh).  With Pd = P z / q the forward
 // output is sum_j Pd_ij v_j, so dV takes Pd^T and dS takes the dropped dP:
-//     dV_j += sum_i Pd_ij dO_i,   dS_ij = P_ij (z_ij dP_ij / (1 - p) - D_i)
+//     dV_j += sum_i Pd_ij dO_i,   dS_ij = P_ij (z_ij dP_ij / q - D_i)
 // (D_i = <dO_i, O_i> is unchanged).  The keep bits are regenerated from the
 // same counters as the forward's.
 template <int D, bool DROP = false>
@@ -235,7 +238,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         mbar_init(&bars->kv_full, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->q_full[s], 1);
-            mbar_init(&bars->q_empty[s], 1);
+            mbar_init(&bars->q_empty[s], 2);  // both MMA issuers read a Q/dO stage
         }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->dp_full, 1);
@@ -244,7 +247,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         mbar_init(&bars->ds_empty, 1);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_empty, 256);
-        mbar_init(&bars->dkdv_full, 1);
+        mbar_init(&bars->dkdv_full, 2);  // dV from issuer 8, dK from issuer 11
         for (int q = 0; q < 4; ++q) mbar_init(&bars->pair[q], 64);
         mbar_init(&bars->dq_staged, 256);
         mbar_init(&bars->dq_free, 1);
@@ -259,9 +262,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp >= 11) {
-        regs_decrease<BWD_REGS_CONTROL>();  // idle warp of the control warpgroup
-    } else if (warp == 9) {
+    if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
         regs_decrease<BWD_REGS_CONTROL>();
         if (lane == 0 && !padding_cta) {
@@ -298,8 +299,8 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             for (int it = max(0, issued - C::QS); it < issued; ++it)
                 mbar_drain(&bars->q_full[it % C::QS], (it / C::QS) & 1);
         }
-    } else if (warp == 8) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 8 || warp == 11) {
+        // ------------------------------------------------------------ MMA issuers
         regs_decrease<BWD_REGS_CONTROL>();
         if (lane == 0 && !padding_cta) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -309,79 +310,88 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             const uint32_t sDS = smem_u32(smem + C::OFF_DS);
             auto sQ = [&](int it) { return smem_u32(smem + C::OFF_Q + (it % C::QS) * C::TILE); };
             auto sdO = [&](int it) { return smem_u32(smem + C::OFF_DO + (it % C::QS) * C::TILE); };
-            auto mma_S = [&](int it) {  // S^T = K Q^T
+            auto q_wait = [&](int it, uint32_t site) {
+                return mbar_wait(&bars->q_full[it % C::QS], (it / C::QS) & 1, g, site);
+            };
+            if (warp == 8) {
+                // S^T(it), dP^T(it), dV(it).  Program order covers the TMEM
+                // reuse of S^T / P^T: S^T(it+1) follows dV(it), which followed
+                // P^T(it) being written, i.e. S^T(it) being read.
+                auto mma_S = [&](int it) {  // S^T = K Q^T
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
-                    mma_ss(tmem + C::T_ST, sdesc_sw128(sK + ko, 16, 1024),
-                           sdesc_sw128(sQ(it) + ko, 16, 1024), id_s, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
+                        mma_ss(tmem + C::T_ST, sdesc_sw128(sK + ko, 16, 1024),
+                               sdesc_sw128(sQ(it) + ko, 16, 1024), id_s, kk > 0);
+                    }
+                    tc_commit(&bars->s_full);
+                };
+                auto mma_dP = [&](int it) {  // dP^T = V dO^T
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
+                        mma_ss(tmem + C::T_DPT, sdesc_sw128(sV + ko, 16, 1024),
+                               sdesc_sw128(sdO(it) + ko, 16, 1024), id_s, kk > 0);
+                    }
+                    tc_commit(&bars->dp_full);
+                };
+                auto mma_dV = [&](int it) {  // dV += P^T dO   (P^T from TMEM)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
+                               sdesc_sw128(sdO(it) + kk * 2048, 16384, 1024), id_kn,
+                               (it > 0 || kk > 0));
+                    tc_commit(&bars->q_empty[it % C::QS]);  // this issuer is done with the stage
+                };
+                bool ok = mbar_wait(&bars->kv_full, 0, g, 22) && q_wait(0, 23);
+                if (ok) {
+                    tc_fence_after();
+                    mma_S(0);
+                    mma_dP(0);
                 }
-                tc_commit(&bars->s_full);
-            };
-            auto mma_dP = [&](int it) {  // dP^T = V dO^T
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
-                    mma_ss(tmem + C::T_DPT, sdesc_sw128(sV + ko, 16, 1024),
-                           sdesc_sw128(sdO(it) + ko, 16, 1024), id_s, kk > 0);
-                }
-                tc_commit(&bars->dp_full);
-            };
-            auto mma_dV = [&](int it) {  // dV += P^T dO   (P^T from TMEM)
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
-                           sdesc_sw128(sdO(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
-            };
-            auto mma_dK_dQ = [&](int it) {  // dK += dS^T Q ; dQ = dS K
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
-                           sdesc_sw128(sQ(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + C::T_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
-                           sdesc_sw128(sK + kk * 2048, 16384, 1024), id_q, kk > 0);
-                tc_commit(&bars->dq_full);
-                tc_commit(&bars->ds_empty);
-                tc_commit(&bars->q_empty[it % C::QS]);
-            };
-            bool ok = mbar_wait(&bars->kv_full, 0, g, 22) &&
-                      mbar_wait(&bars->q_full[0], 0, g, 23);
-            if (ok) {
-                tc_fence_after();
-                mma_S(0);
-                mma_dP(0);
-            }
-            for (int it = 0; ok && it < n_iter; ++it) {
-                const bool more = it + 1 < n_iter;
-                const int s1 = (it + 1) % C::QS;
-                const uint32_t ph1 = ((it + 1) / C::QS) & 1;
-                if (!(ok = mbar_wait(&bars->p_full, it & 1, g, 25))) break;
-                tc_fence_after();
-                mma_dV(it);
-                if (C::EARLY_S && more) {
-                    if (!(ok = mbar_wait(&bars->q_full[s1], ph1, g, 23))) break;
+                for (int it = 0; ok && it < n_iter; ++it) {
+                    const bool more = it + 1 < n_iter;
+                    if (!(ok = mbar_wait(&bars->p_full, it & 1, g, 25))) break;
+                    tc_fence_after();
+                    mma_dV(it);
+                    if (!more) break;
+                    if (!(ok = q_wait(it + 1, 23))) break;
                     tc_fence_after();
                     mma_S(it + 1);
-                }
-                if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 26))) break;
-                if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 27)))
-                    break;
-                tc_fence_after();
-                mma_dK_dQ(it);
-                if (more) {
-                    if (!C::EARLY_S) {
-                        if (!(ok = mbar_wait(&bars->q_full[s1], ph1, g, 23))) break;
-                        tc_fence_after();
-                        mma_S(it + 1);
-                    }
+                    // dP^T(it+1) overwrites dP^T(it): the compute warps must
+                    // have read it (ds_full), and where dQ shares those columns
+                    // (d = 128) they must also have read dQ(it).
+                    if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 26))) break;
                     if (C::DQ_ALIAS && !(ok = mbar_wait(&bars->dq_empty, it & 1, g, 24))) break;
                     tc_fence_after();
                     mma_dP(it + 1);
                 }
+                if (ok) tc_commit(&bars->dkdv_full);
+            } else {
+                // dK(it), dQ(it) from dS(it) in shared memory.
+                bool ok = mbar_wait(&bars->kv_full, 0, g, 37);
+                for (int it = 0; ok && it < n_iter; ++it) {
+                    if (!(ok = q_wait(it, 38))) break;
+                    if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 39))) break;
+                    // dQ(it) overwrites dQ(it-1) in its own columns (d = 64)...
+                    if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 27)))
+                        break;
+                    // ...or dP^T(it), which ds_full shows read (d = 128).
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
+                        mma_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+                               sdesc_sw128(sQ(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // dQ = dS K
+                        mma_ss(tmem + C::T_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                               sdesc_sw128(sK + kk * 2048, 16384, 1024), id_q, kk > 0);
+                    tc_commit(&bars->dq_full);
+                    tc_commit(&bars->ds_empty);
+                    tc_commit(&bars->q_empty[it % C::QS]);
+                }
+                if (ok) tc_commit(&bars->dkdv_full);
             }
-            if (ok) tc_commit(&bars->dkdv_full);
         }
     } else if (warp == 10) {
         // ------------------------------------------------------------ dQ reducer
