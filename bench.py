@@ -36,6 +36,9 @@ UNIT = "TFLOP/s"
 HEADLINE = "b4_h16_n4096_d128"
 DROPOUT_P = 0.1  # attention-dropout rate of the dropout extras (the pages' attn_dropout = 0.1)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's B200 dense (no 2:4 sparsity) BF16 tensor figure, for context only;
+# the roofline uses the measured peak.
+NOMINAL_DENSE_BF16_TFLOPS = 2250.0
 
 
 def load_peaks():
@@ -470,6 +473,7 @@ def run_gpu(args):
                    "l2": "inputs larger than L2 (3 x 67 MB)"},
         "frac_of_bf16_peak": round(per_gpu / peaks["bf16_tflops"], 4),
         "frac_of_bf16_peak_sustained": round(per_gpu / peaks["bf16_tflops_sustained"], 4),
+        "frac_of_nominal_dense_bf16": round(per_gpu / NOMINAL_DENSE_BF16_TFLOPS, 4),
         "roofline": roofline,
         "clocks": clocks,
         "sustained": sustained,
