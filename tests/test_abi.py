@@ -89,3 +89,14 @@ def test_workspace_size_formula(lib):
     assert lib.fa_backward_workspace_bytes(2, 3, 200, 64) == 2 * 3 * 256 * (4 + 4 + 64 * 4)
     assert lib.fa_backward_workspace_bytes(1, 1, 128, 128) == 128 * (8 + 512)
     assert lib.fa_backward_workspace_bytes(1, 1, 0, 64) == 0
+
+
+def test_package_exports_resolve():
+    """Every public name resolves lazily, before and without loading the library."""
+    import importlib
+    import sys
+    for mod in [m for m in sys.modules if m.startswith("io_aware_exact_31_b200")]:
+        del sys.modules[mod]
+    pkg = importlib.import_module("io_aware_exact_31_b200")
+    for name in pkg.__all__:
+        assert getattr(pkg, name) is not None, name
