@@ -64,6 +64,11 @@ def load(path: str | None = None):
                                                      dbl, ip, dbl, u64, u32, vp, vp]
     lib.oracle_attention_backward_dropout.argtypes = [vp, vp, vp, vp, ip, vp, i64, i64, i64, i64,
                                                       i64, dbl, ip, dbl, u64, u32, vp, vp, vp]
+    lib.oracle_attention_forward_dropout_rows.argtypes = [vp, vp, vp, ip, i64, i64, i64, i64, i64,
+                                                          dbl, ip, dbl, u64, u32, vp, i64, vp, vp]
+    lib.oracle_attention_backward_dropout_heads.argtypes = [vp, vp, vp, vp, ip, i64, i64, i64, i64,
+                                                            i64, dbl, ip, dbl, u64, u32, vp, i64,
+                                                            vp, vp, vp]
     lib.oracle_philox4x32_10.argtypes = [vp, vp, vp]
     lib.oracle_philox4x32_10.restype = None
     lib.oracle_dropout_keep_mask.argtypes = [i64, i64, i64, dbl, u64, u32, vp]
@@ -76,7 +81,9 @@ def load(path: str | None = None):
                  "oracle_softmax_merge", "oracle_attention_forward_gqa",
                  "oracle_attention_backward_gqa", "oracle_attention_forward_varlen",
                  "oracle_attention_backward_varlen", "oracle_attention_forward_dropout",
-                 "oracle_attention_backward_dropout", "oracle_dropout_keep_mask"):
+                 "oracle_attention_backward_dropout", "oracle_dropout_keep_mask",
+                 "oracle_attention_forward_dropout_rows",
+                 "oracle_attention_backward_dropout_heads"):
         getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -264,6 +271,48 @@ def attention_backward_dropout(Q, K, V, dO, scale: float, causal: bool, p_drop: 
                                                  int(bool(causal)), float(p_drop), int(seed),
                                                  int(offset), _ptr(dQ), _ptr(dK), _ptr(dV)),
            "oracle_attention_backward_dropout")
+    return dQ, dK, dV
+
+
+def attention_forward_dropout_rows(Q, K, V, scale: float, causal: bool, p_drop: float, seed: int,
+                                   offset: int, rows, lib=None):
+    """Sampled rows (rows[k] = bh*N + i) of attention_forward_dropout (no padding;
+    K/V may have fewer heads).  p_drop = 0: plain attention."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv) = _as_input(Q), _as_input(K), _as_input(V)
+    assert dt == dk == dv and K.shape == V.shape and Q.ndim == 4
+    B, H, N, d = Q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    O = np.empty((rows.size, d), np.float64)
+    LSE = np.empty((rows.size,), np.float64)
+    _check(lib.oracle_attention_forward_dropout_rows(_ptr(Q), _ptr(K), _ptr(V), dt, B, H,
+                                                     K.shape[1], N, d, float(scale),
+                                                     int(bool(causal)), float(p_drop), int(seed),
+                                                     int(offset), _ptr(rows), rows.size, _ptr(O),
+                                                     _ptr(LSE)),
+           "oracle_attention_forward_dropout_rows")
+    return O, LSE
+
+
+def attention_backward_dropout_heads(Q, K, V, dO, scale: float, causal: bool, p_drop: float,
+                                     seed: int, offset: int, heads, lib=None):
+    """attention_backward_dropout restricted to the listed (distinct) query heads
+    bh = b*H + h; other heads' gradients are 0."""
+    lib = lib or load()
+    (Q, dt), (K, dk), (V, dv), (dO, dd) = (_as_input(Q), _as_input(K), _as_input(V),
+                                           _as_input(dO))
+    assert dt == dk == dv == dd and K.shape == V.shape and Q.shape == dO.shape
+    B, H, N, d = Q.shape
+    hs = np.ascontiguousarray(heads, dtype=np.int64)
+    dQ = np.empty((B, H, N, d), np.float64)
+    dK = np.empty(K.shape, np.float64)
+    dV = np.empty(K.shape, np.float64)
+    _check(lib.oracle_attention_backward_dropout_heads(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), dt, B,
+                                                       H, K.shape[1], N, d, float(scale),
+                                                       int(bool(causal)), float(p_drop),
+                                                       int(seed), int(offset), _ptr(hs), hs.size,
+                                                       _ptr(dQ), _ptr(dK), _ptr(dV)),
+           "oracle_attention_backward_dropout_heads")
     return dQ, dK, dV
 
 

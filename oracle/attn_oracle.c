@@ -362,6 +362,47 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
 }
 
 /*
+ * Forward rows with [GQA] heads and [DROP] (no padding): rows[k] = bh * N + i
+ * names query i of query head bh.  As oracle_attention_forward_rows, each
+ * sampled row equals the same row of oracle_attention_forward_dropout.
+ */
+int oracle_attention_forward_dropout_rows(const void *Q, const void *K, const void *V, int dtype,
+                                          int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                          double scale, int causal, double p_drop, uint64_t seed,
+                                          uint32_t offset, const int64_t *rows, int64_t n_rows,
+                                          double *O_rows, double *LSE_rows)
+{
+    struct dropout drop;
+    if (!Q || !K || !V || !rows || !O_rows || !LSE_rows || n_rows < 0 ||
+        bad_shape(B, H, N, d, dtype) || Hkv < 1 || Hkv > H || H % Hkv != 0 ||
+        make_dropout(&drop, p_drop, seed, offset))
+        return -1;
+    for (int64_t k = 0; k < n_rows; ++k)
+        if (rows[k] < 0 || rows[k] >= B * H * N)
+            return -1;
+    const struct dropout *dr = p_drop > 0.0 ? &drop : NULL;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc((size_t)N * sizeof(double));
+        if (!s) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t k = 0; k < n_rows; ++k) {
+            if (!s)
+                continue;
+            const int64_t bh = rows[k] / N, i = rows[k] % N;
+            attention_row(Q, K, V, dtype, N, d, bh * N * d, kv_head(bh, H, Hkv) * N * d, i, scale,
+                          causal, dr, bh, s, O_rows + k * d, LSE_rows + k);
+        }
+        free(s);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
  * Exact gradient of [STD] (with [GQA] heads) for upstream gradient dO, one
  * query head at a time,
  * with the full N x N matrices P, dP and dS materialised ([RECOMP] says only
@@ -383,17 +424,28 @@ int oracle_attention_forward_rows(const void *Q, const void *K, const void *V, i
  * with D, dS, dQ, dK as above (D_i = sum_j P_ij dP_ij still equals
  * <dO_i, O_i>).  dQ is double [B,H,N,d]; dK, dV are double [B,Hkv,N,d].
  */
-int oracle_attention_backward_dropout(const void *Q, const void *K, const void *V,
-                                      const void *dO, int dtype, const int32_t *seqlens,
-                                      int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
-                                      double scale, int causal, double p_drop, uint64_t seed,
-                                      uint32_t offset, double *dQ, double *dK, double *dV)
+static int backward_impl(const void *Q, const void *K, const void *V, const void *dO, int dtype,
+                         const int32_t *seqlens, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                         int64_t d, double scale, int causal, double p_drop, uint64_t seed,
+                         uint32_t offset, const int64_t *heads, int64_t n_heads,
+                         double *dQ, double *dK, double *dV)
 {
     struct dropout drop;
     if (!Q || !K || !V || !dO || !dQ || !dK || !dV || bad_shape(B, H, N, d, dtype) ||
         Hkv < 1 || Hkv > H || H % Hkv != 0 || bad_seqlens(seqlens, B, N) ||
         make_dropout(&drop, p_drop, seed, offset))
         return -1;
+    if (heads) { /* distinct query heads in range */
+        if (n_heads < 0)
+            return -1;
+        for (int64_t a = 0; a < n_heads; ++a) {
+            if (heads[a] < 0 || heads[a] >= B * H)
+                return -1;
+            for (int64_t b = 0; b < a; ++b)
+                if (heads[b] == heads[a])
+                    return -1;
+        }
+    }
     const struct dropout *dr = p_drop > 0.0 ? &drop : NULL;
     double *P = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
     double *dS = (double *)malloc((size_t)N * (size_t)N * sizeof(double));
@@ -411,7 +463,8 @@ int oracle_attention_backward_dropout(const void *Q, const void *K, const void *
     }
     for (int64_t e = 0; e < B * H * N * d; ++e)
         dQ[e] = 0.0;
-    for (int64_t bh = 0; bh < B * H; ++bh) {
+    for (int64_t hi = 0; hi < (heads ? n_heads : B * H); ++hi) {
+        const int64_t bh = heads ? heads[hi] : hi;
         const int64_t base = bh * N * d;                        /* Q, dO, dQ */
         const int64_t kv_base = kv_head(bh, H, Hkv) * N * d;    /* K, V, dK, dV */
         const int64_t N_full = N;
@@ -489,6 +542,37 @@ int oracle_attention_backward_dropout(const void *Q, const void *K, const void *
     free(dS);
     free(Z);
     return 0;
+}
+
+/* The backward of [STD] with [GQA], [PAD] and [DROP]: see backward_impl. */
+int oracle_attention_backward_dropout(const void *Q, const void *K, const void *V,
+                                      const void *dO, int dtype, const int32_t *seqlens,
+                                      int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                                      double scale, int causal, double p_drop, uint64_t seed,
+                                      uint32_t offset, double *dQ, double *dK, double *dV)
+{
+    return backward_impl(Q, K, V, dO, dtype, seqlens, B, H, Hkv, N, d, scale, causal, p_drop,
+                         seed, offset, NULL, 0, dQ, dK, dV);
+}
+
+/*
+ * The same for the listed query heads only (distinct, each bh = b * H + h):
+ * dQ rows of those heads; dK, dV of a K/V head summed over the listed query
+ * heads of its group; everything else 0.  Each head's gradient depends only
+ * on that head, so with one query head per K/V head this equals the full
+ * backward on the listed heads.  For checking large shapes a head at a time.
+ */
+int oracle_attention_backward_dropout_heads(const void *Q, const void *K, const void *V,
+                                            const void *dO, int dtype, int64_t B, int64_t H,
+                                            int64_t Hkv, int64_t N, int64_t d, double scale,
+                                            int causal, double p_drop, uint64_t seed,
+                                            uint32_t offset, const int64_t *heads,
+                                            int64_t n_heads, double *dQ, double *dK, double *dV)
+{
+    if (!heads)
+        return -1;
+    return backward_impl(Q, K, V, dO, dtype, NULL, B, H, Hkv, N, d, scale, causal, p_drop, seed,
+                         offset, heads, n_heads, dQ, dK, dV);
 }
 
 /* Backward with [GQA] heads and [PAD] lengths, no dropout. */

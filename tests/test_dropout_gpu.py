@@ -190,3 +190,46 @@ def test_autograd_wrapper_regenerates_the_mask():
     assert torch.equal(out.detach(), o)
     for a, b in ((q.grad, dq), (k.grad, dk), (v.grad, dv)):
         assert (a.float() - b.float()).abs().max() <= 2e-2 * b.float().abs().max()
+
+
+def test_dropout_forward_full_size_sampled():
+    """The bench's dropout workload (4x16x4096x128, p = 0.1, its seed and
+    offset, the launch bench.py times) on sampled rows of every head."""
+    from io_aware_exact_31_b200.workloads import WORKLOADS, workload_inputs
+    from _parity import sample_rows
+    w = WORKLOADS["b4_h16_n4096_d128"]
+    x = workload_inputs(w, seed=0)
+    q, k, v = (x[n].cuda() for n in ("Q", "K", "V"))
+    o, lse = binding.forward(q, k, v, causal=w.causal, scale=w.scale, dropout_p=0.1, seed=1234,
+                             offset=0)
+    _ok()
+    rows = sample_rows(w.B, w.H, w.N, n_random=2)
+    O_ref, L_ref = oracle.attention_forward_dropout_rows(
+        *(bf16_bits(x[n]) for n in ("Q", "K", "V")), w.scale, w.causal, 0.1, 1234, 0, rows)
+    o_rows = o.reshape(-1, w.d)[torch.from_numpy(rows).cuda()].double().cpu().numpy()
+    l_rows = lse.reshape(-1)[torch.from_numpy(rows).cuda()].double().cpu().numpy()
+    _, eo = o_error(o_rows, O_ref)
+    el = float(np.max(np.abs(l_rows - L_ref)))
+    assert eo <= TOL_O and el <= TOL_LSE, (eo, el)
+
+
+def test_dropout_backward_full_size_sampled_heads():
+    """The bench's dropout backward workload (4x16x2048x64 causal, p = 0.1, its
+    seed) on two whole heads: each head's gradient depends only on that head
+    and, through the keep-mask counter, on its index b*H + h."""
+    from io_aware_exact_31_b200.workloads import WORKLOADS, workload_inputs
+    w = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
+    x = workload_inputs(w, seed=0)
+    q, k, v, do = (x[n].cuda() for n in ("Q", "K", "V", "dO"))
+    o, lse = binding.forward(q, k, v, causal=True, scale=w.scale, dropout_p=0.1, seed=99)
+    dq, dk, dv = binding.backward(q, k, v, o, do, lse, causal=True, scale=w.scale, dropout_p=0.1,
+                                  seed=99)
+    _ok()
+    heads = [0, 2 * w.H + 11]
+    refs = oracle.attention_backward_dropout_heads(
+        *(bf16_bits(x[n]) for n in ("Q", "K", "V", "dO")), w.scale, True, 0.1, 99, 0, heads)
+    for name, g, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), refs):
+        for bh in heads:
+            b, h = divmod(bh, w.H)
+            e = grad_rel_err(g[b, h], r[b, h])
+            assert e <= TOL_GRAD_REL, f"{name} head {bh}: {e:.3e}"

@@ -612,6 +612,35 @@ def pin_dropout_is_unbiased(lib):
     assert np.all(np.abs(runs.mean(axis=0) - O0) <= 6 * se + 1e-12)
 
 
+def pin_dropout_rows_and_heads_match_full(lib):
+    """The sampled variants used at full sizes are bitwise the full oracle:
+    dropout forward rows (GQA, causal) and the backward restricted to heads."""
+    r = _rng(35)
+    B, H, Hkv, N, d = 2, 4, 2, 11, 4
+    Q = r.standard_normal((B, H, N, d))
+    K, V = (r.standard_normal((B, Hkv, N, d)) for _ in range(2))
+    for p_drop in (0.3, 0.0):
+        O, L = oracle.attention_forward_dropout(Q, K, V, 0.6, True, p_drop, 42, 3, lib=lib)
+        rows = np.array([0, 5, N - 1, N + 2, 3 * N + 7, B * H * N - 1])
+        Or, Lr = oracle.attention_forward_dropout_rows(Q, K, V, 0.6, True, p_drop, 42, 3, rows,
+                                                       lib=lib)
+        assert np.array_equal(Or, O.reshape(-1, d)[rows]) and np.array_equal(Lr, L.reshape(-1)[rows])
+    Q, dO, K, V = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    dQ, dK, dV = oracle.attention_backward_dropout(Q, K, V, dO, 0.6, False, 0.25, 7, 1, lib=lib)
+    heads = [5, 2]
+    hq, hk, hv = oracle.attention_backward_dropout_heads(Q, K, V, dO, 0.6, False, 0.25, 7, 1, heads,
+                                                         lib=lib)
+    for t, f in ((hq, dQ), (hk, dK), (hv, dV)):
+        t2, f2 = t.reshape(B * H, N, d), f.reshape(B * H, N, d)
+        for bh in range(B * H):
+            if bh in heads:
+                assert np.array_equal(t2[bh], f2[bh]), bh
+            else:
+                assert not t2[bh].any(), bh
+    with pytest.raises(RuntimeError):
+        oracle.attention_backward_dropout_heads(Q, K, V, dO, 0.6, False, 0.25, 7, 1, [2, 2], lib=lib)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -702,6 +731,8 @@ MUTANTS = {
     "drop_bwd_dP_unmasked": ("ds[j] = dr ? acc * Z[i * N + j] : acc;", "ds[j] = acc;", 0),
     "drop_bwd_dV_undropped": ("const double pd = dr ? P[i * N + j] * Z[i * N + j] : P[i * N + j];",
                               "const double pd = P[i * N + j];", 0),
+    "drop_rows_query_head_for_kv": ("kv_head(bh, H, Hkv) * N * d, i, scale,\n                          causal, dr, bh",
+                                    "bh * N * d, i, scale,\n                          causal, dr, bh", 0),
     "drop_bwd_kv_head": ("Z[i * N + j] = dropout_keep(dr, bh, i, j)",
                          "Z[i * N + j] = dropout_keep(dr, kv_head(bh, H, Hkv), i, j)", 0),
 }
