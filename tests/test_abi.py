@@ -100,3 +100,40 @@ def test_package_exports_resolve():
     pkg = importlib.import_module("io_aware_exact_31_b200")
     for name in pkg.__all__:
         assert getattr(pkg, name) is not None, name
+
+
+def test_extended_entry_points_reject_bad_arguments_without_a_device(lib):
+    """The documented INVALID_ARG / UNSUPPORTED cases of the grouped, padded,
+    dropout, E4M3, no-alloc and self-test entry points, all returned before
+    any device is touched."""
+    INV, UNS = binding.FA_ERR_INVALID_ARG, binding.FA_ERR_UNSUPPORTED
+    a = [16] * 5  # aligned fake pointers: Q, K, V, O, LSE
+
+    # grouped-query: H_kv must divide H
+    assert lib.fa_forward_gqa(*a, 1, 6, 4, 8, 64, 0.125, 0, None) == INV
+    assert lib.fa_forward_gqa(*a, 1, 4, 0, 8, 64, 0.125, 0, None) == INV
+    # padded batches: seqlens must be 4-byte aligned
+    assert lib.fa_forward_varlen(*a, 18, 1, 2, 2, 8, 64, 0.125, 0, None) == INV
+    # dropout: p in [0, 1 - 2^-16]
+    for pd in (1.0, -0.1, float("nan"), 1.0 - 2.0 ** -17):
+        assert lib.fa_forward_dropout(*a, None, 1, 2, 2, 8, 64, 0.125, 0, pd, 1, 0, None) == INV
+    assert lib.fa_forward_dropout(None, *a[1:], None, 1, 2, 2, 8, 64, 0.125, 0, 0.1, 1, 0,
+                                  None) == INV
+    # E4M3: finite positive descales; d = 128 only
+    for ds in (0.0, -1.0, float("nan"), float("inf")):
+        assert lib.fa_forward_fp8(*a, ds, 1.0, 1.0, 1, 2, 2, 8, 128, 0.125, 0, None) == INV
+        assert lib.fa_forward_fp8(*a, 1.0, 1.0, ds, 1, 2, 2, 8, 128, 0.125, 0, None) == INV
+    assert lib.fa_forward_fp8(*a, 1.0, 1.0, 1.0, 1, 2, 2, 8, 64, 0.125, 0, None) == UNS
+    # backward with dropout: bad p, workspace too small
+    p10 = [16] * 10
+    assert lib.fa_backward_dropout(*p10, 1 << 30, None, 1, 2, 2, 8, 64, 0.125, 0, 1.0, 1, 0,
+                                   None) == INV
+    assert lib.fa_backward_dropout(*p10, 16, None, 1, 2, 2, 8, 64, 0.125, 0, 0.1, 1, 0,
+                                   None) == INV
+    # no-alloc backward: problems beyond its built-in array are UNSUPPORTED
+    p9 = [16] * 9
+    assert lib.fa_backward_noalloc(*p9, 64, 16, 4096, 128, 0.088, 1, None) == UNS
+    assert lib.fa_backward_noalloc(None, *p9[1:], 1, 1, 8, 64, 0.125, 0, None) == INV
+    # bounded-wait self-test: limit must be in (0, 1 s]
+    assert lib.fa_selftest_bounded_wait(0, None) == INV
+    assert lib.fa_selftest_bounded_wait(2_000_000_000, None) == INV
