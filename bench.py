@@ -216,6 +216,8 @@ def run_gpu(args):
     sh = stream.cuda_stream
 
     w = WORKLOADS[HEADLINE]
+    if args.only == "fwd" and args.workload:
+        w = WORKLOADS[args.workload]
 
     def fwd_setup(w):
         x = workload_inputs(w, seed=rank)
@@ -279,7 +281,7 @@ def run_gpu(args):
             dist.destroy_process_group()
         return {"metric": METRIC, "value": round(tflops, 1), "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-                "config": {"workload": f"{HEADLINE} fwd", "dropout_p": args.dropout}, "clocks": clocks,
+                "config": {"workload": f"{w.name} fwd", "dropout_p": args.dropout}, "clocks": clocks,
                 "gpu_launches": args.steps}, rank
 
     # ---------------- e2e through the C ABI with host buffers.  Every step
@@ -588,6 +590,8 @@ def main():
                     help="host time of one oracle step in --impl reference")
     ap.add_argument("--only", default=None, choices=[None, "fwd", "bwd"],
                     help="time only the headline forward / the backward (profiler runs)")
+    ap.add_argument("--workload", default=None,
+                    help="workload name of the --only fwd run (default: the headline)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="attention-dropout rate of the --only fwd / --only bwd runs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,

@@ -20,7 +20,8 @@
 //   warps 4-7  softmax warpgroup for tile 1
 //   warp  8    tcgen05.mma issuer; owns the TMEM allocation
 //   warp  9    TMA producer (Q once, then the K/V ring)
-//   warps 10-11 idle (they complete the third warpgroup, which setmaxnreg needs)
+//   warps 10-11 idle (they complete the third warpgroup, which setmaxnreg needs);
+//              at d = 64 they issue the P.V MMAs of tile 0 and tile 1 (below)
 // TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D)
 //   P_t (bf16, two per column) overwrites the first 64 columns of S_t and is
 //   read by the P.V MMA straight from TMEM.
@@ -30,6 +31,16 @@
 // so softmax of tile 0 overlaps the tile-1 GEMMs and vice versa, and the
 // commit that publishes S_t(j) also guarantees PV_t(j-1) is complete, which is
 // when the softmax warps may rescale O_t in place.
+//
+// d = 64 (bf16) leaves 128 TMEM columns free, enough for P in columns of its
+// own: P0 [384,448)  P1 [448,512).  S_t(j+1) then no longer waits for the
+// softmax of block j to finish -- only for its threads to have read S_t(j)
+// (barrier s_free) -- so it is computed while the exponentials of block j
+// run, and the per-tile chain S -> softmax -> P.V -> S is broken.  Three
+// threads issue the MMAs: warp 8 all S_t, warps 10 and 11 the P.V of tile 0
+// and tile 1 (one thread issues an MMA only every ~110-130 clocks whatever
+// its size, and at d = 64 most of the MMAs are small).  The softmax waits for
+// P.V_t(j-1) (barrier pv_done) before it rescales O_t or overwrites P_t.
 #pragma once
 
 #include "philox.cuh"
@@ -67,6 +78,10 @@ struct FwdCfg {
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
     static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
+    // P in its own columns (see the header): d = 64 with bf16 operands.
+    static constexpr bool SEP = (D == 64) && !F8;
+    static constexpr uint32_t TMEM_P0 = 256 + 2 * D, TMEM_P1 = 256 + 2 * D + 64;
+    static_assert(!SEP || TMEM_P1 + 64 <= 512, "P columns exceed TMEM");
 };
 
 struct FwdParams {
@@ -92,7 +107,9 @@ struct FwdBars {
     uint64_t k_full[3], k_empty[3];
     uint64_t v_full[3], v_empty[3];
     uint64_t s_full[2], p_full[2][2], o_full[2];  // p_full[tile][key half]
+    uint64_t s_free[2], pv_done[2];               // separate-P layout only
 };
+static_assert(sizeof(FwdBars) + 8 <= 256, "barrier area");
 
 // DROP: attention dropout (philox.cuh) on the bf16 path; the 1 / (1 - p)
 // factor arrives folded into p.o_scale.
@@ -150,13 +167,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         }
         for (int s = 0; s < C::NV; ++s) {
             mbar_init(&bars->v_full[s], 1);
-            mbar_init(&bars->v_empty[s], 1);
+            mbar_init(&bars->v_empty[s], C::SEP ? 2 : 1);  // SEP: one commit per P.V issuer
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars->s_full[t], 1);
             mbar_init(&bars->p_full[t][0], 128);
             mbar_init(&bars->p_full[t][1], 128);
             mbar_init(&bars->o_full[t], 1);
+            mbar_init(&bars->s_free[t], 128);
+            mbar_init(&bars->pv_done[t], 1);
         }
         fence_barrier_init();
     }
@@ -170,8 +189,42 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
 
     if (warp >= 10) {
-        // idle warps of the control warpgroup
         regs_decrease<FWD_REGS_CONTROL>();
+        if constexpr (C::SEP) {
+            // -------------------------------------------- P.V issuer of tile t
+            const int t = static_cast<int>(warp) - 10;
+            if (lane == 0 && !padding_cta) {
+                const uint32_t idO = idesc_bf16(128, D, false, true);
+                const uint32_t sV = smem_u32(smem + C::OFF_V);
+                const uint32_t tO = tmem + (t == 0 ? C::TMEM_O0 : C::TMEM_O1);
+                const uint32_t tP = tmem + (t == 0 ? C::TMEM_P0 : C::TMEM_P1);
+                bool ok = true;
+                for (int j = 0; ok && j < n_blocks; ++j) {
+                    const int sv = j % C::NV;
+                    if (!(ok = mbar_wait(&bars->v_full[sv], (j / C::NV) & 1, g, 17 + t))) break;
+                    if (j < n_tile[t]) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            if (!(ok = mbar_wait(&bars->p_full[t][h], j & 1, g, 19 + 2 * t + h))) break;
+                            tc_fence_after();
+                            // O_t (+)= P_t V_j for keys [64h, 64h + 64): P from
+                            // TMEM (8 columns per instruction), V MN-major.
+#pragma unroll
+                            for (int i = 0; i < C::PV_PER_HALF; ++i) {
+                                const int kk = h * C::PV_PER_HALF + i;
+                                const uint64_t b = sdesc_sw128(
+                                    sV + sv * C::TILE_BYTES + kk * C::KSTEP * 128, 16384, 1024);
+                                mma_ts(tO, tP + kk * 8, b, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                            }
+                        }
+                        if (!ok) break;
+                        tc_commit(&bars->pv_done[t]);
+                    }
+                    // Both issuers release V(j), whether or not this tile used it.
+                    tc_commit(&bars->v_empty[sv]);
+                }
+            }
+        }
     } else if (warp == 9) {
         regs_decrease<FWD_REGS_CONTROL>();
         // ------------------------------------------------------------ TMA producer
@@ -261,51 +314,73 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 }
             };
 
-            bool ok = mbar_wait(&bars->q_full, 0, g, 3) && mbar_wait(&bars->k_full[0], 0, g, 4);
-            if (ok) {
-                tc_fence_after();
-                issue_S(0, 0);
-                tc_commit(&bars->s_full[0]);
-                issue_S(1, 0);
-                tc_commit(&bars->s_full[1]);
-                tc_commit(&bars->k_empty[0]);
-            }
-            for (int j = 1; ok && j <= n_blocks; ++j) {
-                // Finish block j-1 (P.V) for both tiles, then start block j (S).
-                // Each wait sits right before the first MMA that needs it, and
-                // V(j-1)'s slot is released right after its last P.V.
-                const int sv = (j - 1) % C::NV;
-                const uint32_t phv = ((j - 1) / C::NV) & 1;
-                const int sk = j % C::NK;
-                const uint32_t phk = (j / C::NK) & 1;
-                const bool more = j < n_blocks;
-                bool k_ready = false;
-                if (!(ok = mbar_wait(&bars->v_full[sv], phv, g, 6))) break;
-                tc_fence_after();
+            bool ok = mbar_wait(&bars->q_full, 0, g, 3);
+            if constexpr (C::SEP) {
+                // S issuer: S_t(j) as soon as K(j) is in and the softmax threads
+                // of tile t have read S_t(j - 1) into registers.
+                for (int j = 0; ok && j < n_blocks; ++j) {
+                    const int sk = j % C::NK;
+                    if (!(ok = mbar_wait(&bars->k_full[sk], (j / C::NK) & 1, g, 5))) break;
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (j - 1 < n_tile[t]) {
-                        if (!(ok = mbar_wait(&bars->p_full[t][0], (j - 1) & 1, g, 7 + t))) break;
-                        tc_fence_after();
-                        issue_PV_half(t, sv, 0, j > 1);
-                        if (!(ok = mbar_wait(&bars->p_full[t][1], (j - 1) & 1, g, 13 + t))) break;
-                        tc_fence_after();
-                        issue_PV_half(t, sv, 1, true);
-                        if (j == n_tile[t]) tc_commit(&bars->o_full[t]);
-                    }
-                    if (t == 1) tc_commit(&bars->v_empty[sv]);
-                    if (more && j < n_tile[t]) {
-                        if (!k_ready) {
-                            if (!(ok = mbar_wait(&bars->k_full[sk], phk, g, 5))) break;
+                    for (int t = 0; t < 2; ++t) {
+                        if (j < n_tile[t]) {
+                            if (j > 0 && !(ok = mbar_wait(&bars->s_free[t], (j - 1) & 1, g, 15 + t)))
+                                break;
                             tc_fence_after();
-                            k_ready = true;
+                            issue_S(t, sk);
+                            tc_commit(&bars->s_full[t]);
                         }
-                        issue_S(t, sk);
-                        tc_commit(&bars->s_full[t]);
                     }
+                    if (!ok) break;
+                    tc_commit(&bars->k_empty[sk]);
                 }
-                if (!ok) break;
-                if (more) tc_commit(&bars->k_empty[sk]);
+            } else {  // P over S: one issuer for every MMA
+                ok = ok && mbar_wait(&bars->k_full[0], 0, g, 4);
+                if (ok) {
+                    tc_fence_after();
+                    issue_S(0, 0);
+                    tc_commit(&bars->s_full[0]);
+                    issue_S(1, 0);
+                    tc_commit(&bars->s_full[1]);
+                    tc_commit(&bars->k_empty[0]);
+                }
+                for (int j = 1; ok && j <= n_blocks; ++j) {
+                    // Finish block j-1 (P.V) for both tiles, then start block j (S).
+                    // Each wait sits right before the first MMA that needs it, and
+                    // V(j-1)'s slot is released right after its last P.V.
+                    const int sv = (j - 1) % C::NV;
+                    const uint32_t phv = ((j - 1) / C::NV) & 1;
+                    const int sk = j % C::NK;
+                    const uint32_t phk = (j / C::NK) & 1;
+                    const bool more = j < n_blocks;
+                    bool k_ready = false;
+                    if (!(ok = mbar_wait(&bars->v_full[sv], phv, g, 6))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        if (j - 1 < n_tile[t]) {
+                            if (!(ok = mbar_wait(&bars->p_full[t][0], (j - 1) & 1, g, 7 + t))) break;
+                            tc_fence_after();
+                            issue_PV_half(t, sv, 0, j > 1);
+                            if (!(ok = mbar_wait(&bars->p_full[t][1], (j - 1) & 1, g, 13 + t))) break;
+                            tc_fence_after();
+                            issue_PV_half(t, sv, 1, true);
+                            if (j == n_tile[t]) tc_commit(&bars->o_full[t]);
+                        }
+                        if (t == 1) tc_commit(&bars->v_empty[sv]);
+                        if (more && j < n_tile[t]) {
+                            if (!k_ready) {
+                                if (!(ok = mbar_wait(&bars->k_full[sk], phk, g, 5))) break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_S(t, sk);
+                            tc_commit(&bars->s_full[t]);
+                        }
+                    }
+                    if (!ok) break;
+                    if (more) tc_commit(&bars->k_empty[sk]);
+                }
             }
         }
     } else {
@@ -317,6 +392,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         const int q = q0 + t * FWD_BM + row;       // query index
         const uint32_t tS = tmem_addr(tmem, lane_base, t == 0 ? C::TMEM_S0 : C::TMEM_S1);
         const uint32_t tO = tmem_addr(tmem, lane_base, t == 0 ? C::TMEM_O0 : C::TMEM_O1);
+        // Where P goes: over the first columns of S_t, or its own columns (SEP).
+        const uint32_t tP =
+            C::SEP ? tmem_addr(tmem, lane_base, t == 0 ? C::TMEM_P0 : C::TMEM_P1) : tS;
         const float sl2 = p.scale_log2;
         float m_used = -INFINITY;  // running row max, log2 units of scaled scores
         float l = 0.f;             // running row sum of exp2(s*sl2 - m_used) (for LSE)
@@ -339,6 +417,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
             tmem_ld_wait();
             reg_fence<128>(sr);
+            if constexpr (C::SEP) {
+                // S_t is in registers: the tensor core may overwrite it with S_t(j+1).
+                tc_fence_before();
+                mbar_arrive(&bars->s_free[t]);
+            }
             float s[128];
 #pragma unroll
             for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
@@ -376,19 +459,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             // exp2(-inf - 0) = 0 instead of NaN.
             const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
             // Rescale O_t in place when this row's max moved (rare after the
-            // first blocks).  PV_t(j-1) is complete: it was issued before S_t(j).
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            // first blocks).  PV_t(j-1) must be complete: with P over S it was
+            // issued before S_t(j), whose commit we waited for; with P in its
+            // own columns the softmax waits for pv_done first (below).
+            auto rescale_O = [&]() {
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + c * 32, o);
-                    tmem_ld_wait();
-                    reg_fence<32>(o);
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + c * 32, o);
+                        tmem_ld_wait();
+                        reg_fence<32>(o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tO + c * 32, o);
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tO + c * 32, o);
+                    }
                 }
-            }
+            };
+            if constexpr (!C::SEP) rescale_O();
             l *= alpha;
             lr *= alpha;
             // p = exp2(s * scale_log2 - m), rounded to bf16 for the P.V product.
@@ -437,14 +526,26 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                         }
                     }
                 }
-                if constexpr (F8) tmem_st16(tS + h * C::P_COLS_HALF, pk);
-                else tmem_st32(tS + h * C::P_COLS_HALF, pk);
+                if constexpr (C::SEP) {
+                    if (h == 0) {
+                        // P_t and O_t are free once P.V_t(j-1) has completed.
+                        if (j > 0) {
+                            if (!(ok = mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, g, 23 + t)))
+                                break;
+                            tc_fence_after();
+                        }
+                        rescale_O();
+                    }
+                }
+                if constexpr (F8) tmem_st16(tP + h * C::P_COLS_HALF, pk);
+                else tmem_st32(tP + h * C::P_COLS_HALF, pk);
                 // Release this half of P: the tensor core starts on keys
                 // [64h, 64h + 64) while the other half is still being computed.
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&bars->p_full[t][h]);
             }
+            if (!ok) break;
             {
                 const float2 e = __fadd2_rn(__fadd2_rn(ae[0], ae[1]), __fadd2_rn(ae[2], ae[3]));
                 const float2 r = __fadd2_rn(__fadd2_rn(ar[0], ar[1]), __fadd2_rn(ar[2], ar[3]));
@@ -461,7 +562,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
                 p.LSE[static_cast<size_t>(bh) * p.N + q] = 0.f;
             }
-        } else if (ok && mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t)) {
+        } else if (ok && (C::SEP ? mbar_wait_warp(&bars->pv_done[t], (nt - 1) & 1, g, 25 + t)
+                                 : mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t))) {
             tc_fence_after();
             const bool real = q < len;  // padding rows of a partly padded tile get zeros
             const float inv_l = real ? p.o_scale / lr : 0.f;
