@@ -499,7 +499,10 @@ def run_gpu(args):
                          "peak_basis": f"16 ex2/clk/SM x {sm_count} SMs x sampled sm_mhz"}
 
     # ---------------- context only: torch's own SDPA kernels on the same box
-    extra["context_torch_sdpa"] = torch_sdpa_context(torch, w, w5, stream, args, max_ranks)
+    try:
+        extra["context_torch_sdpa"] = torch_sdpa_context(torch, w, w5, stream, args, max_ranks)
+    except ImportError as e:  # a torch without torch.nn.attention
+        extra["context_torch_sdpa"] = {"unavailable": f"{type(e).__name__}: {e}"}
 
     traffic = recorded_traffic()
     achieved = per_gpu
