@@ -457,6 +457,81 @@ def run_gpu(args):
                                   "fwd_tflops": round(w5.fwd_flops / (msfd * 1e-3) / 1e12, 1),
                                   "bwd_tflops": round(w5.bwd_flops / (msbd * 1e-3) / 1e12, 1)}}
 
+    # ---------------- extra: grouped-query attention and padded batches on the
+    # headline shape (forward) and on the 4x16x2048x64 causal shape (forward +
+    # backward).  FLOPs count each query head against its keys (grouped-query)
+    # and the real tokens of each batch only (padding).
+    def gen(shape, seed_):
+        g_ = torch.Generator(device="cpu").manual_seed(seed_)
+        return torch.randn(*shape, generator=g_).to(torch.bfloat16).cuda()
+
+    def padded_flops(lens, H_, d_, causal_):
+        return sum(4.0 * H_ * n_ * n_ * d_ * (0.5 if causal_ else 1.0) for n_ in lens)
+
+    def time_steps(fn):
+        for _ in range(args.warmup):
+            fn()
+        return max_ranks(time_region(fn, args.steps, stream, barrier)) / args.steps
+
+    hkv = 2
+    qg = gen((w.B, w.H, w.N, w.d), 10 + rank)
+    kg, vg = gen((w.B, hkv, w.N, w.d), 11 + rank), gen((w.B, hkv, w.N, w.d), 12 + rank)
+    og = torch.empty_like(qg)
+    lg = torch.empty(w.B, w.H, w.N, device="cuda", dtype=torch.float32)
+    msg = time_steps(lambda: binding.forward(qg, kg, vg, causal=w.causal, scale=w.scale, out=og,
+                                             lse=lg, stream=stream))
+    extra[w.name + "_gqa"] = {"pass": "fwd", "H_kv": hkv, "ms": round(msg, 4),
+                              "tflops": round(w.fwd_flops / (msg * 1e-3) / 1e12, 1),
+                              "frac_of_bf16_peak": round(w.fwd_flops / (msg * 1e-3) / 1e12 /
+                                                         peaks["bf16_tflops"], 4)}
+    del kg, vg
+    lens = [w.N, 3 * w.N // 4, w.N // 2, w.N // 4][:w.B]
+    kp, vp = gen((w.B, w.H, w.N, w.d), 13 + rank), gen((w.B, w.H, w.N, w.d), 14 + rank)
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    msp = time_steps(lambda: binding.forward(qg, kp, vp, causal=w.causal, scale=w.scale, out=og,
+                                             lse=lg, stream=stream, seqlens=sl))
+    fp = padded_flops(lens, w.H, w.d, w.causal)
+    extra[w.name + "_padded"] = {"pass": "fwd", "seqlens": lens, "ms": round(msp, 4),
+                                 "tflops_real_tokens": round(fp / (msp * 1e-3) / 1e12, 1),
+                                 "frac_of_bf16_peak": round(fp / (msp * 1e-3) / 1e12 /
+                                                            peaks["bf16_tflops"], 4)}
+    del qg, kp, vp, og, lg, sl
+
+    hkv5 = 4
+    q5g, do5g = gen((w5.B, w5.H, w5.N, w5.d), 20 + rank), gen((w5.B, w5.H, w5.N, w5.d), 21 + rank)
+    k5g, v5g = gen((w5.B, hkv5, w5.N, w5.d), 22 + rank), gen((w5.B, hkv5, w5.N, w5.d), 23 + rank)
+    o5g, l5g = binding.forward(q5g, k5g, v5g, causal=True, scale=w5.scale)
+    dq5g, dk5g, dv5g = torch.empty_like(q5g), torch.empty_like(k5g), torch.empty_like(v5g)
+    msfg = time_steps(lambda: binding.forward(q5g, k5g, v5g, causal=True, scale=w5.scale,
+                                              out=o5g, lse=l5g, stream=stream))
+    msbg = time_steps(lambda: binding.backward(q5g, k5g, v5g, o5g, do5g, l5g, causal=True,
+                                               scale=w5.scale, dq=dq5g, dk=dk5g, dv=dv5g,
+                                               workspace=ws, stream=stream))
+    k5p, v5p = gen((w5.B, w5.H, w5.N, w5.d), 24 + rank), gen((w5.B, w5.H, w5.N, w5.d), 25 + rank)
+    lens5 = [w5.N, 3 * w5.N // 4, w5.N // 2, w5.N // 4][:w5.B]
+    sl5 = torch.tensor(lens5, dtype=torch.int32, device="cuda")
+    o5p, l5p = binding.forward(q5g, k5p, v5p, causal=True, scale=w5.scale, seqlens=sl5)
+    dk5p, dv5p = torch.empty_like(k5p), torch.empty_like(v5p)
+    msfp = time_steps(lambda: binding.forward(q5g, k5p, v5p, causal=True, scale=w5.scale,
+                                              out=o5p, lse=l5p, stream=stream, seqlens=sl5))
+    msbp = time_steps(lambda: binding.backward(q5g, k5p, v5p, o5p, do5g, l5p, causal=True,
+                                               scale=w5.scale, dq=dq5g, dk=dk5p, dv=dv5p,
+                                               workspace=ws, stream=stream, seqlens=sl5))
+    st, site = binding.check_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {site:#x}")
+    fp5 = padded_flops(lens5, w5.H, w5.d, True)
+    extra[w5.name]["gqa"] = {"H_kv": hkv5, "fwd_ms": round(msfg, 4), "bwd_ms": round(msbg, 4),
+                             "fwd_tflops": round(w5.fwd_flops / (msfg * 1e-3) / 1e12, 1),
+                             "bwd_tflops": round(w5.bwd_flops / (msbg * 1e-3) / 1e12, 1)}
+    extra[w5.name]["padded"] = {"seqlens": lens5, "fwd_ms": round(msfp, 4),
+                                "bwd_ms": round(msbp, 4),
+                                "fwd_tflops_real_tokens": round(fp5 / (msfp * 1e-3) / 1e12, 1),
+                                "bwd_tflops_real_tokens": round(2.5 * fp5 / (msbp * 1e-3) / 1e12,
+                                                                1)}
+    del q5g, do5g, k5g, v5g, o5g, l5g, dq5g, dk5g, dv5g, k5p, v5p, o5p, l5p, dk5p, dv5p, sl5
+    torch.cuda.empty_cache()
+
     # ---------------- extra: the two small workloads, each launch timed alone
     # after a 256 MB write that evicts L2 (their inputs would otherwise stay
     # resident); median over the launches
