@@ -137,3 +137,18 @@ def test_extended_entry_points_reject_bad_arguments_without_a_device(lib):
     # bounded-wait self-test: limit must be in (0, 1 s]
     assert lib.fa_selftest_bounded_wait(0, None) == INV
     assert lib.fa_selftest_bounded_wait(2_000_000_000, None) == INV
+
+
+def test_python_entry_points_reject_host_tensors():
+    """No CPU fallback: every Python entry point refuses tensors that are not
+    contiguous bf16 CUDA tensors before anything is launched."""
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.forward(q, q, q)
+    with pytest.raises(ValueError):
+        binding.backward(q, q, q, q, q, torch.zeros(1, 2, 8))
+    with pytest.raises(ValueError):
+        binding.attention(q, q, q)
+    with pytest.raises(ValueError):
+        binding.forward(q.float(), q.float(), q.float())
