@@ -302,7 +302,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     } else if (warp == 8 || warp == 11) {
         // ------------------------------------------------------------ MMA issuers
         regs_decrease<BWD_REGS_CONTROL>();
-        if (lane == 0 && !padding_cta) {
+        if (!padding_cta) {  // the whole warp; one elected lane issues
             const uint32_t id_s = idesc_bf16(128, 128, false, false);  // S^T, dP^T
             const uint32_t id_kn = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
             const uint32_t id_q = idesc_bf16(128, D, true, true);      // dQ (A, B MN-major)
@@ -311,7 +311,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             auto sQ = [&](int it) { return smem_u32(smem + C::OFF_Q + (it % C::QS) * C::TILE); };
             auto sdO = [&](int it) { return smem_u32(smem + C::OFF_DO + (it % C::QS) * C::TILE); };
             auto q_wait = [&](int it, uint32_t site) {
-                return mbar_wait(&bars->q_full[it % C::QS], (it / C::QS) & 1, g, site);
+                return mbar_wait_warp(&bars->q_full[it % C::QS], (it / C::QS) & 1, g, site);
             };
             if (warp == 8) {
                 // S^T(it), dP^T(it), dV(it).  Program order covers the TMEM
@@ -321,29 +321,29 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
-                        mma_ss(tmem + C::T_ST, sdesc_sw128(sK + ko, 16, 1024),
+                        mma_ss_w(tmem + C::T_ST, sdesc_sw128(sK + ko, 16, 1024),
                                sdesc_sw128(sQ(it) + ko, 16, 1024), id_s, kk > 0);
                     }
-                    tc_commit(&bars->s_full);
+                    tc_commit_w(&bars->s_full);
                 };
                 auto mma_dP = [&](int it) {  // dP^T = V dO^T
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
-                        mma_ss(tmem + C::T_DPT, sdesc_sw128(sV + ko, 16, 1024),
+                        mma_ss_w(tmem + C::T_DPT, sdesc_sw128(sV + ko, 16, 1024),
                                sdesc_sw128(sdO(it) + ko, 16, 1024), id_s, kk > 0);
                     }
-                    tc_commit(&bars->dp_full);
+                    tc_commit_w(&bars->dp_full);
                 };
                 auto mma_dV = [&](int it) {  // dV += P^T dO   (P^T from TMEM)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
+                        mma_ts_w(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
                                sdesc_sw128(sdO(it) + kk * 2048, 16384, 1024), id_kn,
                                (it > 0 || kk > 0));
-                    tc_commit(&bars->q_empty[it % C::QS]);  // this issuer is done with the stage
+                    tc_commit_w(&bars->q_empty[it % C::QS]);  // this issuer is done with the stage
                 };
-                bool ok = mbar_wait(&bars->kv_full, 0, g, 22) && q_wait(0, 23);
+                bool ok = mbar_wait_warp(&bars->kv_full, 0, g, 22) && q_wait(0, 23);
                 if (ok) {
                     tc_fence_after();
                     mma_S(0);
@@ -351,7 +351,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
                 }
                 for (int it = 0; ok && it < n_iter; ++it) {
                     const bool more = it + 1 < n_iter;
-                    if (!(ok = mbar_wait(&bars->p_full, it & 1, g, 25))) break;
+                    if (!(ok = mbar_wait_warp(&bars->p_full, it & 1, g, 25))) break;
                     tc_fence_after();
                     mma_dV(it);
                     if (!more) break;
@@ -361,36 +361,36 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
                     // dP^T(it+1) overwrites dP^T(it): the compute warps must
                     // have read it (ds_full), and where dQ shares those columns
                     // (d = 128) they must also have read dQ(it).
-                    if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 26))) break;
-                    if (C::DQ_ALIAS && !(ok = mbar_wait(&bars->dq_empty, it & 1, g, 24))) break;
+                    if (!(ok = mbar_wait_warp(&bars->ds_full, it & 1, g, 26))) break;
+                    if (C::DQ_ALIAS && !(ok = mbar_wait_warp(&bars->dq_empty, it & 1, g, 24))) break;
                     tc_fence_after();
                     mma_dP(it + 1);
                 }
-                if (ok) tc_commit(&bars->dkdv_full);
+                if (ok) tc_commit_w(&bars->dkdv_full);
             } else {
                 // dK(it), dQ(it) from dS(it) in shared memory.
-                bool ok = mbar_wait(&bars->kv_full, 0, g, 37);
+                bool ok = mbar_wait_warp(&bars->kv_full, 0, g, 37);
                 for (int it = 0; ok && it < n_iter; ++it) {
                     if (!(ok = q_wait(it, 38))) break;
-                    if (!(ok = mbar_wait(&bars->ds_full, it & 1, g, 39))) break;
+                    if (!(ok = mbar_wait_warp(&bars->ds_full, it & 1, g, 39))) break;
                     // dQ(it) overwrites dQ(it-1) in its own columns (d = 64)...
-                    if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, g, 27)))
+                    if (!C::DQ_ALIAS && it > 0 && !(ok = mbar_wait_warp(&bars->dq_empty, (it - 1) & 1, g, 27)))
                         break;
                     // ...or dP^T(it), which ds_full shows read (d = 128).
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
-                        mma_ss(tmem + C::T_DK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+                        mma_ss_w(tmem + C::T_DK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
                                sdesc_sw128(sQ(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)  // dQ = dS K
-                        mma_ss(tmem + C::T_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                        mma_ss_w(tmem + C::T_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
                                sdesc_sw128(sK + kk * 2048, 16384, 1024), id_q, kk > 0);
-                    tc_commit(&bars->dq_full);
-                    tc_commit(&bars->ds_empty);
-                    tc_commit(&bars->q_empty[it % C::QS]);
+                    tc_commit_w(&bars->dq_full);
+                    tc_commit_w(&bars->ds_empty);
+                    tc_commit_w(&bars->q_empty[it % C::QS]);
                 }
-                if (ok) tc_commit(&bars->dkdv_full);
+                if (ok) tc_commit_w(&bars->dkdv_full);
             }
         }
     } else if (warp == 10) {

@@ -193,7 +193,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         if constexpr (C::SEP) {
             // -------------------------------------------- P.V issuer of tile t
             const int t = static_cast<int>(warp) - 10;
-            if (lane == 0 && !padding_cta) {
+            if (!padding_cta) {  // the whole warp; one elected lane issues
                 const uint32_t idO = idesc_bf16(128, D, false, true);
                 const uint32_t sV = smem_u32(smem + C::OFF_V);
                 const uint32_t tO = tmem + (t == 0 ? C::TMEM_O0 : C::TMEM_O1);
@@ -201,27 +201,29 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 bool ok = true;
                 for (int j = 0; ok && j < n_blocks; ++j) {
                     const int sv = j % C::NV;
-                    if (!(ok = mbar_wait(&bars->v_full[sv], (j / C::NV) & 1, g, 17 + t))) break;
+                    if (!(ok = mbar_wait_warp(&bars->v_full[sv], (j / C::NV) & 1, g, 17 + t))) break;
                     if (j < n_tile[t]) {
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            if (!(ok = mbar_wait(&bars->p_full[t][h], j & 1, g, 19 + 2 * t + h))) break;
+                            if (!(ok = mbar_wait_warp(&bars->p_full[t][h], j & 1, g, 19 + 2 * t + h))) break;
                             tc_fence_after();
                             // O_t (+)= P_t V_j for keys [64h, 64h + 64): P from
                             // TMEM (8 columns per instruction), V MN-major.
+                            // descriptor of this V stage; k-steps advance its
+                            // address field (16-byte units, no carry: < 256 KB)
+                            const uint64_t b0 = sdesc_sw128(sV + sv * C::TILE_BYTES, 16384, 1024);
 #pragma unroll
                             for (int i = 0; i < C::PV_PER_HALF; ++i) {
                                 const int kk = h * C::PV_PER_HALF + i;
-                                const uint64_t b = sdesc_sw128(
-                                    sV + sv * C::TILE_BYTES + kk * C::KSTEP * 128, 16384, 1024);
-                                mma_ts(tO, tP + kk * 8, b, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                                mma_ts_w(tO, tP + kk * 8, b0 + (kk * C::KSTEP * 128 >> 4), idO,
+                                         (j > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
                         if (!ok) break;
-                        tc_commit(&bars->pv_done[t]);
+                        tc_commit_w(&bars->pv_done[t]);
                     }
                     // Both issuers release V(j), whether or not this tile used it.
-                    tc_commit(&bars->v_empty[sv]);
+                    tc_commit_w(&bars->v_empty[sv]);
                 }
             }
         }
@@ -278,7 +280,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         regs_decrease<FWD_REGS_CONTROL>();
-        if (lane == 0 && !padding_cta) {
+        if (!padding_cta) {  // the whole warp; one elected lane issues
             // S = Q K^T (K-major A, B); O += P V (V MN-major)
             const uint32_t idS = F8 ? idesc_e4m3(128, FWD_BN, false) : idesc_bf16(128, FWD_BN, false, false);
             const uint32_t idO = F8 ? idesc_e4m3(128, D, true) : idesc_bf16(128, D, false, true);
@@ -295,8 +297,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
                     const uint64_t a = sdesc_sw128(sQ + t * C::TILE_BYTES + koff, 16, 1024);
                     const uint64_t b = sdesc_sw128(sK + s * C::TILE_BYTES + koff, 16, 1024);
-                    if constexpr (F8) mma_ss_f8(tS[t], a, b, idS, kk > 0);
-                    else mma_ss(tS[t], a, b, idS, kk > 0);
+                    if constexpr (F8) mma_ss_f8_w(tS[t], a, b, idS, kk > 0);
+                    else mma_ss_w(tS[t], a, b, idS, kk > 0);
                 }
             };
             // O_t (+)= P_t V_j for keys [64h, 64h + 64): P from TMEM (8 columns
@@ -309,40 +311,40 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     const int kk = h * C::PV_PER_HALF + i;
                     const uint64_t b = sdesc_sw128(sV + s * C::TILE_BYTES + kk * C::KSTEP * 128,
                                                    16384, 1024);
-                    if constexpr (F8) mma_ts_f8(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
-                    else mma_ts(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
+                    if constexpr (F8) mma_ts_f8_w(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
+                    else mma_ts_w(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
                 }
             };
 
-            bool ok = mbar_wait(&bars->q_full, 0, g, 3);
+            bool ok = mbar_wait_warp(&bars->q_full, 0, g, 3);
             if constexpr (C::SEP) {
                 // S issuer: S_t(j) as soon as K(j) is in and the softmax threads
                 // of tile t have read S_t(j - 1) into registers.
                 for (int j = 0; ok && j < n_blocks; ++j) {
                     const int sk = j % C::NK;
-                    if (!(ok = mbar_wait(&bars->k_full[sk], (j / C::NK) & 1, g, 5))) break;
+                    if (!(ok = mbar_wait_warp(&bars->k_full[sk], (j / C::NK) & 1, g, 5))) break;
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         if (j < n_tile[t]) {
-                            if (j > 0 && !(ok = mbar_wait(&bars->s_free[t], (j - 1) & 1, g, 15 + t)))
+                            if (j > 0 && !(ok = mbar_wait_warp(&bars->s_free[t], (j - 1) & 1, g, 15 + t)))
                                 break;
                             tc_fence_after();
                             issue_S(t, sk);
-                            tc_commit(&bars->s_full[t]);
+                            tc_commit_w(&bars->s_full[t]);
                         }
                     }
                     if (!ok) break;
-                    tc_commit(&bars->k_empty[sk]);
+                    tc_commit_w(&bars->k_empty[sk]);
                 }
             } else {  // P over S: one issuer for every MMA
-                ok = ok && mbar_wait(&bars->k_full[0], 0, g, 4);
+                ok = ok && mbar_wait_warp(&bars->k_full[0], 0, g, 4);
                 if (ok) {
                     tc_fence_after();
                     issue_S(0, 0);
-                    tc_commit(&bars->s_full[0]);
+                    tc_commit_w(&bars->s_full[0]);
                     issue_S(1, 0);
-                    tc_commit(&bars->s_full[1]);
-                    tc_commit(&bars->k_empty[0]);
+                    tc_commit_w(&bars->s_full[1]);
+                    tc_commit_w(&bars->k_empty[0]);
                 }
                 for (int j = 1; ok && j <= n_blocks; ++j) {
                     // Finish block j-1 (P.V) for both tiles, then start block j (S).
@@ -354,32 +356,32 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     const uint32_t phk = (j / C::NK) & 1;
                     const bool more = j < n_blocks;
                     bool k_ready = false;
-                    if (!(ok = mbar_wait(&bars->v_full[sv], phv, g, 6))) break;
+                    if (!(ok = mbar_wait_warp(&bars->v_full[sv], phv, g, 6))) break;
                     tc_fence_after();
 #pragma unroll
                     for (int t = 0; t < 2; ++t) {
                         if (j - 1 < n_tile[t]) {
-                            if (!(ok = mbar_wait(&bars->p_full[t][0], (j - 1) & 1, g, 7 + t))) break;
+                            if (!(ok = mbar_wait_warp(&bars->p_full[t][0], (j - 1) & 1, g, 7 + t))) break;
                             tc_fence_after();
                             issue_PV_half(t, sv, 0, j > 1);
-                            if (!(ok = mbar_wait(&bars->p_full[t][1], (j - 1) & 1, g, 13 + t))) break;
+                            if (!(ok = mbar_wait_warp(&bars->p_full[t][1], (j - 1) & 1, g, 13 + t))) break;
                             tc_fence_after();
                             issue_PV_half(t, sv, 1, true);
-                            if (j == n_tile[t]) tc_commit(&bars->o_full[t]);
+                            if (j == n_tile[t]) tc_commit_w(&bars->o_full[t]);
                         }
-                        if (t == 1) tc_commit(&bars->v_empty[sv]);
+                        if (t == 1) tc_commit_w(&bars->v_empty[sv]);
                         if (more && j < n_tile[t]) {
                             if (!k_ready) {
-                                if (!(ok = mbar_wait(&bars->k_full[sk], phk, g, 5))) break;
+                                if (!(ok = mbar_wait_warp(&bars->k_full[sk], phk, g, 5))) break;
                                 tc_fence_after();
                                 k_ready = true;
                             }
                             issue_S(t, sk);
-                            tc_commit(&bars->s_full[t]);
+                            tc_commit_w(&bars->s_full[t]);
                         }
                     }
                     if (!ok) break;
-                    if (more) tc_commit(&bars->k_empty[sk]);
+                    if (more) tc_commit_w(&bars->k_empty[sk]);
                 }
             }
         }

@@ -365,6 +365,54 @@ __device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
 }
 
+// Warp-collective forms of the MMA and commit above.  The whole warp, converged,
+// executes the call; elect.sync inside the instruction block picks one lane
+// (the same lane every time in a fully converged warp, so the commit tracks
+// the MMAs that lane issued).  Issued this way a single warp sends
+// back-to-back M = 128, N = 128, K = 16 MMAs every ~94 (shared-memory A) /
+// ~105 (TMEM A) clocks and N = 256 ones at the tensor core's full rate,
+// against ~140 clocks per instruction from a lane-0 branch of a diverged warp
+// (microbenchmark on B200, 148 SMs, one issuing warp per SM).
+#define FA_ELECT_MMA(kind, aop)                                                        \
+    "{\n\t.reg .pred p, e;\n\t"                                                          \
+    "elect.sync _|e, 0xffffffff;\n\t"                                                    \
+    "setp.ne.b32 p, %4, 0;\n\t"                                                          \
+    "@e tcgen05.mma.cta_group::1.kind::" kind " [%0], " aop ", %2, %3, p;\n\t}"
+
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(FA_ELECT_MMA("f16", "%1")::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc),
+                 "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(FA_ELECT_MMA("f16", "[%1]")::"r"(d_tmem), "r"(a_tmem), "l"(b_desc),
+                 "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_ss_f8_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(FA_ELECT_MMA("f8f6f4", "%1")::"r"(d_tmem), "l"(a_desc), "l"(b_desc),
+                 "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_ts_f8_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(FA_ELECT_MMA("f8f6f4", "[%1]")::"r"(d_tmem), "r"(a_tmem), "l"(b_desc),
+                 "r"(idesc), "r"(accumulate));
+}
+
+// Warp-collective tc_commit (the elected lane is the one that issued the MMAs).
+__device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
 // Load 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives
 // lane (lane_base + t).  The warp may only touch its own 32-lane quarter
 // (warp_id % 4).  Results are valid only after tmem_ld_wait().
