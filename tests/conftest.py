@@ -24,3 +24,28 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the largest errors each parity test saw (raw max |O - O_ref|,
+    the same beyond the bf16 rounding of O_ref, |LSE| error, gradient
+    relative errors), and write them as JSON to $FA_PARITY_RECORD if set."""
+    mod = sys.modules.get("_parity")
+    rec = getattr(mod, "RECORD", None) if mod else None
+    if not rec:
+        return
+    cols = ["o_raw", "o_beyond_bf16", "fp8_err_over_band", "lse", "grad_rel", "dQ", "dK", "dV", "rows_checked",
+            "heads_checked"]
+    tr = terminalreporter
+    tr.write_sep("-", "parity errors per test (max over the test's checks)")
+    tr.write_line("test | " + " | ".join(cols))
+    for test in sorted(rec):
+        r = rec[test]
+        tr.write_line(test + " | " + " | ".join(
+            ("%.3e" % r[c] if c not in ("rows_checked", "heads_checked") else "%d" % r[c])
+            if c in r else "-" for c in cols))
+    path = os.environ.get("FA_PARITY_RECORD")
+    if path:
+        import json
+        with open(path, "w") as f:
+            json.dump(rec, f, indent=1, sort_keys=True)

@@ -1,4 +1,5 @@
 """Backward parity: CUDA path (through the C ABI) vs the fp64 oracle."""
+import numpy as np
 import pytest
 import torch
 
@@ -24,8 +25,15 @@ def test_multi_block(d):
 
 
 def test_b4_h16_n2048_d64_causal_sampled_heads():
+    """The full backward workload; the oracle checks 16 of its 64 heads: the
+    first and last head of every batch (the first and last CTAs of each
+    batch's key blocks) and eight more drawn at random."""
     w = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
-    check_backward(w.B, w.H, w.N, w.d, w.causal, heads=[(0, 0), (1, 7), (3, 15)])
+    ends = [(b, h) for b in range(w.B) for h in (0, w.H - 1)]
+    rest = [(b, h) for b in range(w.B) for h in range(1, w.H - 1)]
+    r = np.random.default_rng(2)
+    pick = [rest[i] for i in sorted(r.choice(len(rest), size=8, replace=False))]
+    check_backward(w.B, w.H, w.N, w.d, w.causal, heads=ends + pick)
 
 
 def test_autograd_wrapper_matches_raw():

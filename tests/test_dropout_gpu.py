@@ -22,7 +22,7 @@ import oracle
 from io_aware_exact_31_b200 import binding
 from io_aware_exact_31_b200.workloads import bf16_bits
 
-from _parity import TOL_GRAD_REL, TOL_LSE, TOL_O, grad_rel_err, o_error
+from _parity import TOL_GRAD_REL, TOL_LSE, TOL_O, grad_rel_err, o_error, record
 
 pytestmark = pytest.mark.gpu
 
@@ -133,6 +133,7 @@ def test_dropout_parity(B, H, Hkv, N, p, seqlens, causal, d):
                                                     seqlens=seqlens)
     _, eo = o_error(o.double().cpu().numpy(), O_ref)
     el = float(np.max(np.abs(lse.double().cpu().numpy() - L_ref)))
+    record(lse=el)
     assert eo <= TOL_O and el <= TOL_LSE, (eo, el)
     refs = oracle.attention_backward_dropout(*bits, scale, causal, p, seed, offset,
                                              seqlens=seqlens)
@@ -210,6 +211,7 @@ def test_dropout_forward_full_size_sampled():
     l_rows = lse.reshape(-1)[torch.from_numpy(rows).cuda()].double().cpu().numpy()
     _, eo = o_error(o_rows, O_ref)
     el = float(np.max(np.abs(l_rows - L_ref)))
+    record(lse=el)
     assert eo <= TOL_O and el <= TOL_LSE, (eo, el)
 
 

@@ -22,7 +22,7 @@ import torch
 import oracle
 from io_aware_exact_31_b200 import binding
 
-from _parity import TOL_LSE, bf16_rounding_distance
+from _parity import TOL_LSE, bf16_rounding_distance, record
 
 pytestmark = pytest.mark.gpu
 
@@ -116,5 +116,8 @@ def test_fp8_forward_full_size_sampled():
         band = (1.1 * (2.0 ** -4 * (wts @ dev) + 2.0 ** -10 * wts.max() * dev.sum(0)) +
                 bf16_rounding_distance(O_ref[k]))
         worst = max(worst, float(np.max(np.abs(o_rows[k] - O_ref[k]) / band)))
+    el = float(np.max(np.abs(l_rows - L_ref)))
+    record(o_raw=float(np.max(np.abs(o_rows - O_ref))), fp8_err_over_band=worst, lse=el,
+           rows_checked=rows.size)
     assert worst <= 1.0, f"error/band max {worst:.3f}"
-    assert float(np.max(np.abs(l_rows - L_ref))) <= TOL_LSE
+    assert el <= TOL_LSE

@@ -13,7 +13,7 @@ import oracle
 from io_aware_exact_31_b200 import binding
 from io_aware_exact_31_b200.workloads import bf16_bits
 
-from _parity import TOL_GRAD_REL, TOL_LSE, TOL_O, grad_rel_err, o_error
+from _parity import TOL_GRAD_REL, TOL_LSE, TOL_O, grad_rel_err, o_error, record
 
 pytestmark = pytest.mark.gpu
 
@@ -73,6 +73,7 @@ def test_random_configuration_matches_oracle(case):
                                                     seqlens=seqlens)
     _, eo = o_error(o.double().cpu().numpy(), O_ref)
     el = float(np.max(np.abs(lse.double().cpu().numpy() - L_ref)))
+    record(lse=el)
     assert eo <= TOL_O and el <= TOL_LSE, f"max|dO|={eo:.3e} max|dLSE|={el:.3e}"
     refs = oracle.attention_backward_dropout(*bits, scale, causal, p, seed, offset,
                                              seqlens=seqlens)

@@ -11,7 +11,7 @@ import oracle
 from io_aware_exact_31_b200 import binding
 from io_aware_exact_31_b200.workloads import bf16_bits
 
-from _parity import TOL_GRAD_REL, TOL_LSE, TOL_O, grad_rel_err, o_error
+from _parity import TOL_GRAD_REL, TOL_LSE, TOL_O, grad_rel_err, o_error, record
 
 pytestmark = pytest.mark.gpu
 
@@ -39,6 +39,7 @@ def test_gqa_forward_backward(H, Hkv, causal, N, d):
     O_ref, L_ref = oracle.attention_forward_gqa(*bits[:3], scale, causal)
     _, eo = o_error(o.double().cpu().numpy(), O_ref)
     el = float(np.max(np.abs(lse.double().cpu().numpy() - L_ref)))
+    record(lse=el)
     assert eo <= TOL_O and el <= TOL_LSE, (eo, el)
     refs = oracle.attention_backward_gqa(*bits, scale, causal)
     for name, gr, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), refs):
