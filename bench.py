@@ -87,7 +87,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, period: float = 0.002):
+    def __init__(self, device_index: int, period: float = 0.0):
         self.dev, self.period = device_index, period
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = None
@@ -117,7 +117,8 @@ class ClockSampler:
                 except Exception as e:  # noqa: BLE001
                     self.error = str(e)
                     return
-                self._stop.wait(self.period)
+                if self.period > 0:
+                    self._stop.wait(self.period)
 
         self._thr = threading.Thread(target=loop, daemon=True)
         self._thr.start()
@@ -147,7 +148,9 @@ class ClockSampler:
                     "samples": 0, "note": self.error}
         return {"sm_mhz": statistics.median(self.samples), "sm_min_mhz": min(self.samples),
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples), "source": "NVML, 2 ms period"}
+                "samples": len(self.samples),
+                "source": "NVML, back-to-back queries" if self.period <= 0
+                else f"NVML, {self.period * 1e3:g} ms period"}
 
 
 def dist_setup(args):
@@ -550,6 +553,26 @@ def run_gpu(args):
         ts = sorted(a.elapsed_time(b) for a, b in evs)
         return ts[len(ts) // 2]
 
+    def host_latency_us(a, n=200):
+        """Host-side cost of one call through the C ABI: the enqueue alone
+        (fa_forward returning) and the call plus a stream synchronise (the
+        latency a caller that waits for the result sees); medians."""
+        enq, full = [], []
+        for _ in range(n):
+            t0 = time.perf_counter()
+            launch_fwd(a)
+            t1 = time.perf_counter()
+            stream.synchronize()
+            t2 = time.perf_counter()
+            enq.append(t1 - t0)
+            full.append(t2 - t0)
+        enq.sort()
+        full.sort()
+        return {"enqueue_us": round(enq[n // 2] * 1e6, 2),
+                "call_and_sync_us": round(full[n // 2] * 1e6, 2), "calls": n,
+                "note": "host wall clock around the ctypes call (Python overhead included); "
+                        "tensor maps come from the library's cache after the first call"}
+
     for name in ("tiny_n256_d64", "transformer_h8_n1024_d64_causal"):
         ws_ = WORKLOADS[name]
         _, bs_, as_ = fwd_setup(ws_)
@@ -558,7 +581,8 @@ def run_gpu(args):
         msf_ = max_ranks(flushed_ms(lambda: launch_fwd(as_), max(args.steps, 20)))
         extra[name] = {"pass": "fwd", "ms": round(msf_, 4), "l2": "flushed before each launch",
                        "tflops": round(ws_.fwd_flops / (msf_ * 1e-3) / 1e12, 2),
-                       "statistic": "median of single launches"}
+                       "statistic": "median of single launches",
+                       "latency_us": host_latency_us(as_)}
         del bs_, as_
     del flush
     torch.cuda.empty_cache()
@@ -587,6 +611,18 @@ def run_gpu(args):
                 "traffic": traffic, "algorithmic_bytes": w.fwd_bytes,
                 "algorithmic_flops": w.fwd_flops}
 
+    # The backward of the 4x16x2048x64 causal workload: three launches (pre,
+    # main, dQ finalise) timed together by CUDA events; the main kernel's share
+    # of that time comes from the committed ncu launch list.
+    roofline_bwd = {"bound": "tensor", "kernel": "fa_bwd_pre + fa_bwd_main_kernel<64> + "
+                    "fa_bwd_dq (one backward)", "workload": w5.name,
+                    "achieved": round(w5.bwd_flops / (msb * 1e-3) / 1e12, 1),
+                    "peak": peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16_tflops (burst)",
+                    "unit": "TFLOP/s",
+                    "frac": round(w5.bwd_flops / (msb * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                    "traffic": None, "algorithmic_bytes": w5.bwd_bytes,
+                    "algorithmic_flops": w5.bwd_flops}
+
     result = {
         "metric": METRIC, "value": round(tflops, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -599,6 +635,7 @@ def run_gpu(args):
         "frac_of_bf16_peak_sustained": round(per_gpu / peaks["bf16_tflops_sustained"], 4),
         "frac_of_nominal_dense_bf16": round(per_gpu / NOMINAL_DENSE_BF16_TFLOPS, 4),
         "roofline": roofline,
+        "roofline_bwd": roofline_bwd,
         "clocks": clocks,
         "sustained": sustained,
         "e2e": {"value": round(w.fwd_flops * world / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
@@ -733,6 +770,108 @@ def oracle_sample(target_s: float, step_rows: int | None = None):
     return flops_per_row * rows / dt / 1e12, dt, rows, threads
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo where it exists)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine() or "unknown"
+
+
+def oracle_baseline(c3_seconds: float):
+    """The fp64 oracle timed on this host's cores, workload by workload:
+    the 256-token and 8-head 1024-token forwards in full (all threads and one
+    thread), the headline forward on a random row sample (about c3_seconds),
+    the 16k causal forward on a stated row sample with its full time
+    extrapolated, and the 4x16x2048x64 causal forward and backward in full.
+    Returns the cpu_baseline object; its value is the headline's sample."""
+    import numpy as np
+
+    import oracle
+    from io_aware_exact_31_b200.workloads import WORKLOADS, bf16_bits, workload_inputs
+
+    threads = oracle.num_threads()
+    per = {}
+
+    def bits(w):
+        return {n: bf16_bits(t) for n, t in workload_inputs(w).items()}
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    for name in ("tiny_n256_d64", "transformer_h8_n1024_d64_causal"):
+        w = WORKLOADS[name]
+        b = bits(w)
+
+        def run(w=w, b=b):
+            oracle.attention_forward(b["Q"], b["K"], b["V"], w.scale, w.causal)
+
+        run()  # first touch of the inputs and the thread pool
+        t_all = timed(run)
+        oracle.set_num_threads(1)
+        try:
+            t_one = timed(run)
+        finally:
+            oracle.set_num_threads(threads)
+        per[name + " fwd"] = {"run": "full", "seconds": round(t_all, 4),
+                              "tflops": w.fwd_flops / t_all / 1e12,
+                              "seconds_1_thread": round(t_one, 4),
+                              "tflops_1_thread": w.fwd_flops / t_one / 1e12}
+
+    tf3, dt3, rows3, _ = oracle_sample(c3_seconds)
+    w3 = WORKLOADS[HEADLINE]
+    per[HEADLINE + " fwd"] = {
+        "run": f"row sample: {rows3} random query rows of {w3.B * w3.H * w3.N}, seed 1",
+        "seconds": round(dt3, 3), "tflops": tf3,
+        "full_seconds_extrapolated": round(w3.fwd_flops / (tf3 * 1e12), 1)}
+
+    # 16k causal: every head's rows 0 and N-1 and 254 random rows (seed 1).
+    # A causal row i costs (i + 1) key visits, so the full time is the
+    # sample's time scaled by all rows' key visits over the sample's.
+    w4 = WORKLOADS["h16_n16384_d128_causal_x2"]
+    b4 = bits(w4)
+    rng = np.random.default_rng(1)
+    rows4 = []
+    for bh in range(w4.B * w4.H):
+        rnd = rng.choice(np.arange(1, w4.N - 1), size=254, replace=False)
+        rows4.extend(bh * w4.N + i for i in sorted({0, w4.N - 1, *(int(v) for v in rnd)}))
+    rows4 = np.array(rows4, np.int64)
+    dt4 = timed(lambda: oracle.attention_forward_rows(b4["Q"], b4["K"], b4["V"], w4.scale,
+                                                      w4.causal, rows4))
+    visits_sample = float(np.sum(rows4 % w4.N + 1))
+    visits_all = float(w4.B * w4.H) * w4.N * (w4.N + 1) / 2
+    t4_full = dt4 * visits_all / visits_sample
+    per[w4.name + " fwd"] = {
+        "run": f"row sample, extrapolated: rows 0, N-1 and 254 random rows (seed 1) of each "
+               f"of the {w4.B * w4.H} heads ({rows4.size} rows); full time = sample time x "
+               f"(all rows' key visits / the sample's)",
+        "seconds": round(dt4, 3), "full_seconds_extrapolated": round(t4_full, 1),
+        "tflops": w4.fwd_flops / t4_full / 1e12}
+    del b4
+
+    w5 = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
+    b5 = bits(w5)
+    dt5f = timed(lambda: oracle.attention_forward(b5["Q"], b5["K"], b5["V"], w5.scale, True))
+    dt5b = timed(lambda: oracle.attention_backward(b5["Q"], b5["K"], b5["V"], b5["dO"],
+                                                   w5.scale, True))
+    per[w5.name + " fwd"] = {"run": "full", "seconds": round(dt5f, 3),
+                             "tflops": w5.fwd_flops / dt5f / 1e12}
+    per[w5.name + " bwd"] = {"run": "full", "seconds": round(dt5b, 3),
+                             "tflops": w5.bwd_flops / dt5b / 1e12}
+    return {"value": tf3, "unit": UNIT, "cores": threads, "cpu_model": cpu_model(),
+            "kind": "oracle",
+            "sample": f"{rows3} random query rows of {HEADLINE} (forward, fp64, {dt3:.1f} s on "
+                      f"{threads} threads)",
+            "per_workload": per}
+
+
 def run_reference(args):
     world, rank, _ = dist_setup(args)
     if rank != 0:
@@ -780,8 +919,9 @@ def main():
                     help="workload name of the --only fwd run (default: the headline)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="attention-dropout rate of the --only fwd / --only bwd runs")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0,
-                    help="target host time of the oracle CPU-baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="target host time of the oracle's headline row sample (0: no CPU "
+                         "baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -795,10 +935,7 @@ def main():
     world, rank, _ = dist_setup(args)
     cpu = None
     if world == 1 and rank == 0 and args.cpu_seconds > 0:
-        tf, dt, rows, threads = oracle_sample(args.cpu_seconds)
-        cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"{rows} random query rows of {HEADLINE} (forward, fp64, "
-                         f"{dt:.1f} s on {threads} threads)"}
+        cpu = oracle_baseline(args.cpu_seconds)
     res, rank = run_gpu(args)
     if rank == 0:
         res["cpu_baseline"] = cpu
