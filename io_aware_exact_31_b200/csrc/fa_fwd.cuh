@@ -516,7 +516,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                         }
                     } else {
                         pk[i] = pack_bf16x2(pe.x, pe.y);
-                        ar[i % 4] = __fadd2_rn(ar[i % 4], unpack_bf16x2(pk[i]));
+                        add_bf16x2_f32(ar[i % 4], pk[i]);
                         if constexpr (DROP) {
                             // Dropped weights leave the P.V product but stay in
                             // both row sums (the softmax is of undropped scores).

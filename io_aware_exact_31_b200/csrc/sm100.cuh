@@ -115,6 +115,41 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
         if (globaltimer() - t0 > FA_WAIT_TIMEOUT_NS) return;
 }
 
+// Bounded wait until a global counter reaches `target` (acquire).  Gives up,
+// returning false, when the CTA aborts, when another CTA has already recorded
+// an error in the device error word (so that CTAs queued behind a failed one
+// do not each wait out the full limit), or after the wall-clock limit.
+__device__ __forceinline__ bool wait_counter(const int* cnt, int target, const Guard& g,
+                                             uint32_t site) {
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        if (v >= target) return true;
+        if (*g.abort_flag) return false;
+        if (g.err && *reinterpret_cast<volatile uint32_t*>(g.err) != 0u) {
+            *g.abort_flag = 1;
+            return false;
+        }
+        if (globaltimer() - t0 > FA_WAIT_TIMEOUT_NS) {
+            guard_fail(g, DEV_TIMEOUT_BASE + site);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+
+// counter += 1 with release semantics at GPU scope.
+__device__ __forceinline__ void counter_release_add(int* cnt) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(cnt) : "memory");
+}
+
+// Order this thread's generic-proxy and async-proxy (bulk copy) accesses to
+// global memory with respect to each other.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Warp-collective wait: every lane polls (each acquires the barrier), then the
 // outcome is made uniform and the warp reconverged, so the .sync.aligned
 // tcgen05 instructions that follow are executed by all 32 lanes together.
@@ -491,6 +526,19 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// acc.x += the low bf16 of w, acc.y += its high bf16: one mixed-precision add
+// (bf16 operand, f32 accumulator, round to nearest) per half.  The result is
+// bit-identical to widening each half to f32 and adding, without the two
+// integer operations the widening costs.
+__device__ __forceinline__ void add_bf16x2_f32(float2& acc, uint32_t w) {
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "r"(w));
 }
 
 // Three-input maximum (one instruction on sm_100).
