@@ -135,7 +135,8 @@ fa_status fa_forward_fp8(const void *Q8, const void *K8, const void *V8, void *O
 /*
  * Device workspace fa_backward needs, in bytes (0 on invalid shapes).  It holds
  * D_i = <dO_i, O_i>, LSE in base-2 units and the fp32 dQ accumulator, each
- * padded to a multiple of 128 rows per head.
+ * padded to a multiple of 128 rows per head, and one int32 counter per
+ * 128-row query block (used by fa_backward_deterministic).
  */
 size_t fa_backward_workspace_bytes(int B, int H, int N, int d);
 
@@ -196,6 +197,30 @@ fa_status fa_backward_dropout(const void *Q, const void *K, const void *V, const
                               cudaStream_t stream);
 
 /*
+ * fa_backward_dropout with a run-to-run reproducible dQ.  The pages call the
+ * method "exact and deterministic" (systems-analysis.info "FlashAttention-2
+ * (VI)", performance section).  dK and dV are always bit-reproducible (each is
+ * summed inside one CTA); dQ_i is a sum over key blocks, which the other entry
+ * points add into an fp32 accumulator in whatever order the key-block CTAs
+ * reach it, so its last bits may vary between runs.  Here the additions into
+ * each 128-row dQ block are made in ascending key-block order: a CTA waits
+ * (bounded) until every lower key block of the same head has added its part,
+ * adds its own and publishes a per-block counter in the workspace.  Results
+ * are bitwise identical across runs with the same inputs, grid and device.
+ *   Arguments: as fa_backward_dropout (dropout_p = 0 and seqlens = NULL for the
+ *     plain backward; H_kv = H for multi-head attention).
+ *   Errors: as fa_backward_dropout; a wait that gives up is reported through
+ *     fa_check_device_error as FA_ERR_TIMEOUT.
+ */
+fa_status fa_backward_deterministic(const void *Q, const void *K, const void *V, const void *O,
+                                    const void *dO, const float *LSE, void *dQ, void *dK,
+                                    void *dV, void *workspace, size_t workspace_bytes,
+                                    const int *seqlens, int B, int H, int H_kv, int N, int d,
+                                    float scale, int causal, float dropout_p,
+                                    unsigned long long seed, unsigned int offset,
+                                    cudaStream_t stream);
+
+/*
  * Size of the device array fa_backward_noalloc uses as its workspace (64 MiB).
  * Every GPU on which this library's device code is loaded holds one such
  * array until the process exits, whether or not fa_backward_noalloc is called.
@@ -217,7 +242,10 @@ fa_status fa_backward_dropout(const void *Q, const void *K, const void *V, const
  *     (e.g. B*H = 64 heads of N = 2048, d = 64 need 33 MiB and fit).
  *   First call on each device: looks up the array's device address and sets
  *     kernel attributes (host-side set-up only); make that first call before
- *     any stream capture.
+ *     any stream capture.  The address is kept for the life of the process,
+ *     like the device error word's, so it assumes the device's primary
+ *     context lives as long: after cudaDeviceReset on a device, do not call
+ *     this library on that device again.
  *   Sharing: every call on a device uses the same array.  Calls whose kernels
  *     can overlap on the GPU (other streams, other host threads) race on it
  *     and give undefined results; serialise them, e.g. on one stream.  Each

@@ -21,7 +21,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 EXPORTS = ("fa_forward", "fa_forward_gqa", "fa_forward_varlen", "fa_forward_dropout",
            "fa_forward_fp8", "fa_backward_workspace_bytes",
            "fa_backward", "fa_backward_gqa", "fa_backward_varlen", "fa_backward_dropout",
-           "fa_backward_noalloc",
+           "fa_backward_deterministic", "fa_backward_noalloc",
            "fa_check_device_error", "fa_selftest_bounded_wait", "fa_status_str", "fa_version")
 
 # Size of the library's built-in workspace used by fa_backward_noalloc.
@@ -70,6 +70,8 @@ def load_library(path: str | None = None):
     lib.fa_backward_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, i, i, i, i,
                                         i, f, i, f, u64, u32, vp]
     lib.fa_backward_dropout.restype = i
+    lib.fa_backward_deterministic.argtypes = list(lib.fa_backward_dropout.argtypes)
+    lib.fa_backward_deterministic.restype = i
     lib.fa_forward_fp8.argtypes = [vp, vp, vp, vp, vp, f, f, f, i, i, i, i, i, f, i, vp]
     lib.fa_forward_fp8.restype = i
     lib.fa_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
@@ -194,10 +196,12 @@ def forward_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None, stream=None,
              seqlens: torch.Tensor | None = None, dropout_p: float = 0.0, seed: int = 0,
-             offset: int = 0):
+             offset: int = 0, deterministic: bool = False):
     """dQ, dK, dV of <O, dO> (scores recomputed from the saved LSE).  With K/V
     of fewer heads, dK/dV are summed over each group of query heads.  The
-    dropout arguments must be those of the forward call."""
+    dropout arguments must be those of the forward call.  deterministic=True
+    adds the key blocks' dQ parts in a fixed order (fa_backward_deterministic),
+    so that dQ is bitwise reproducible from run to run."""
     B, H, N, d, Hkv = _check_kv_heads(q, k, v)
     _check_qkv(q, o, do)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
@@ -213,7 +217,10 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
             lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
             workspace.numel() * workspace.element_size(), sl, B, H, Hkv, N, d, scale,
             int(bool(causal)))
-    if dropout_p:
+    if deterministic:
+        st = lib.fa_backward_deterministic(*args, float(dropout_p), int(seed), int(offset),
+                                           _stream_handle(stream))
+    elif dropout_p:
         st = lib.fa_backward_dropout(*args, float(dropout_p), int(seed), int(offset),
                                      _stream_handle(stream))
     else:

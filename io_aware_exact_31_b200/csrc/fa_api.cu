@@ -312,6 +312,35 @@ fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const
                : FA_ERR_CUDA;
 }
 
+fa_status fa_backward_deterministic(const void* Q, const void* K, const void* V, const void* O,
+                                    const void* dO, const float* LSE, void* dQ, void* dK,
+                                    void* dV, void* workspace, size_t workspace_bytes,
+                                    const int* seqlens, int B, int H, int H_kv, int N, int d,
+                                    float scale, int causal, float dropout_p,
+                                    unsigned long long seed, unsigned int offset,
+                                    cudaStream_t stream) {
+    DropoutParams drop;
+    bool on = false;
+    fa_status st = make_dropout(dropout_p, seed, offset, &drop, &on);
+    if (st != FA_OK) return st;
+    if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace)
+        return FA_ERR_INVALID_ARG;
+    if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_INVALID_ARG;
+    const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return FA_ERR_INVALID_ARG;
+    if ((st = check_shape(B, H, N, d, scale)) != FA_OK) return st;
+    if ((st = check_heads(H, H_kv)) != FA_OK) return st;
+    if (workspace_bytes < bwd_workspace_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+    DeviceState* ds = current_device(&st);
+    if (!ds) return st;
+    if (!ensure_bwd_attributes(ds, d, on)) return FA_ERR_CUDA;
+    return bwd_launch(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, H_kv, N, d, seqlens,
+                      scale, causal, ds->err, on ? &drop : nullptr, stream, true)
+               ? FA_OK
+               : FA_ERR_CUDA;
+}
+
 fa_status fa_backward_varlen(const void* Q, const void* K, const void* V, const void* O,
                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                              void* workspace, size_t workspace_bytes, const int* seqlens, int B,

@@ -49,9 +49,15 @@ constexpr uint32_t BWD_REGS_CONTROL = 88;
 inline size_t round_up_128(int n) { return (static_cast<size_t>(n) + 127) / 128 * 128; }
 
 // Workspace: [D: BH*Npad f32][LSE2: BH*Npad f32][dQacc: BH*Npad*d f32]
+//            [dQ block counters: BH*Npad/128 int32, padded to 256 B]
+// The counters order the dQ additions in the deterministic mode.
+inline size_t bwd_counter_bytes(int B, int H, int N) {
+    const size_t n = static_cast<size_t>(B) * H * (round_up_128(N) / 128);
+    return (n * 4 + 255) / 256 * 256;
+}
 inline size_t bwd_workspace_bytes(int B, int H, int N, int d) {
     const size_t rows = static_cast<size_t>(B) * H * round_up_128(N);
-    return rows * 4 * 2 + rows * static_cast<size_t>(d) * 4;
+    return rows * 4 * 2 + rows * static_cast<size_t>(d) * 4 + bwd_counter_bytes(B, H, N);
 }
 
 template <int D>
@@ -97,6 +103,7 @@ struct BwdParams {
     int H, group;        // query heads per batch; query heads per K/V head
     int Hkv, n_kv_heads; // K/V heads per batch; B * Hkv
     const int* seqlens;  // [B] real tokens per batch (device), or null
+    int* dq_count;       // [BH, Npad/128] dQ block counters (deterministic mode), or null
     float scale, scale_log2;
     int causal;
     uint32_t* err;
@@ -111,9 +118,12 @@ __global__ void __launch_bounds__(256)
 fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                   const float* __restrict__ LSE, float* __restrict__ Dvec,
                   float* __restrict__ LSE2, float* __restrict__ dQacc, int N, int Npad,
-                  long long rows_pad, const int* __restrict__ seqlens, int H) {
+                  long long rows_pad, const int* __restrict__ seqlens, int H,
+                  int* __restrict__ dq_count, long long n_count) {
     constexpr int TPR = D / 8;  // threads per row, 8 bf16 (16 B) each
     const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (long long c = tid; c < n_count; c += static_cast<long long>(gridDim.x) * blockDim.x)
+        dq_count[c] = 0;
     const int sub = threadIdx.x % TPR;
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x / TPR;
     for (long long r = tid / TPR; r < rows_pad; r += stride) {
@@ -398,15 +408,35 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         regs_decrease<BWD_REGS_CONTROL>();
         if (lane == 0) {
             tma_prefetch_desc(&mapdQacc);
+            // Deterministic mode: the additions into one dQ block are made in
+            // ascending key-block order.  Before adding, wait until the block's
+            // counter equals this CTA's key block (every earlier key block of
+            // the same head has added and published); after the addition has
+            // fully completed, publish by incrementing the counter.  Only CTAs
+            // with a lower grid index are waited for (both CTA orders put a
+            // head's lower key blocks first), so the waits always end.
+            const bool det = p.dq_count != nullptr;
             for (int it = 0; it < n_iter; ++it) {
                 if (!mbar_wait(&bars->dq_staged, it & 1, g, 28)) break;
                 const int q0 = q_block0(it), bh = q_head(it);
+                int* cnt = det ? p.dq_count + static_cast<size_t>(bh) * p.n_q_blocks + q0 / BWD_BM
+                               : nullptr;
+                if (det) {
+                    if (!wait_counter(cnt, kb, g, 31)) break;
+                    fence_proxy_async_global();
+                }
 #pragma unroll
                 for (int b = 0; b < D / 32; ++b)
                     tma_reduce_add_3d(&mapdQacc, smem + C::OFF_DQ + b * 16384, b * 32, q0, bh);
                 bulk_commit_group();
                 bulk_wait_read_all();
                 mbar_arrive(&bars->dq_free);
+                if (det) {
+                    bulk_wait_all();
+                    __threadfence();
+                    fence_proxy_async_global();
+                    counter_release_add(cnt);
+                }
             }
             bulk_wait_all();
         }
@@ -642,18 +672,20 @@ template <int D, bool DROP>
 bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                   const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
                   int Hkv, int N, const int* seqlens, float scale, int causal, uint32_t* err,
-                  const DropoutParams& drop, cudaStream_t stream) {
+                  const DropoutParams& drop, bool deterministic, cudaStream_t stream) {
     const int Npad = static_cast<int>(round_up_128(N));
     const long long rows_pad = static_cast<long long>(B) * H * Npad;
     float* Dvec = static_cast<float*>(workspace);
     float* LSE2 = Dvec + rows_pad;
     float* dQacc = LSE2 + rows_pad;
+    int* dq_count = reinterpret_cast<int*>(dQacc + rows_pad * D);
+    const long long n_count = deterministic ? rows_pad / 128 : 0;
     {
         const long long threads = rows_pad * (D / 8);
         const int blocks = static_cast<int>(std::min<long long>((threads + 255) / 256, 148LL * 16));
         fa_bwd_pre_kernel<D><<<blocks, 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, Dvec,
-            LSE2, dQacc, N, Npad, rows_pad, seqlens, H);
+            LSE2, dQacc, N, Npad, rows_pad, seqlens, H, dq_count, n_count);
         if (cudaGetLastError() != cudaSuccess) return false;
     }
     {
@@ -678,6 +710,7 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         p.Hkv = Hkv;
         p.n_kv_heads = B * Hkv;
         p.seqlens = seqlens;
+        p.dq_count = deterministic ? dq_count : nullptr;
         p.scale = scale;
         p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
         p.causal = causal ? 1 : 0;
@@ -704,12 +737,13 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
 inline bool bwd_launch(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                        const float* LSE, void* dQ, void* dK, void* dV, void* workspace, int B, int H,
                        int Hkv, int N, int d, const int* seqlens, float scale, int causal,
-                       uint32_t* err, const DropoutParams* drop, cudaStream_t stream) {
+                       uint32_t* err, const DropoutParams* drop, cudaStream_t stream,
+                       bool deterministic = false) {
     const DropoutParams none{};
     const DropoutParams& dp = drop ? *drop : none;
 #define FA_BWD_LAUNCH(DD, DR)                                                                    \
     bwd_launch_t<DD, DR>(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, B, H, Hkv, N, seqlens, scale, \
-                         causal, err, dp, stream)
+                         causal, err, dp, deterministic, stream)
     if (d == 128) return drop ? FA_BWD_LAUNCH(128, true) : FA_BWD_LAUNCH(128, false);
     return drop ? FA_BWD_LAUNCH(64, true) : FA_BWD_LAUNCH(64, false);
 #undef FA_BWD_LAUNCH

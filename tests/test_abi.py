@@ -31,6 +31,20 @@ def test_header_declares_expected_entry_points():
     assert set(binding.EXPORTS) <= set(names), names
 
 
+def test_noalloc_limit_matches_the_header():
+    """The binding's copy of the no-allocation backward's array size is the
+    header's FA_BACKWARD_NOALLOC_MAX_SCRATCH_BYTES."""
+    with open(os.path.join(ROOT, "include", "fa.h")) as f:
+        m = re.search(r"#define\s+FA_BACKWARD_NOALLOC_MAX_SCRATCH_BYTES\s+\(([^)]*)\)", f.read())
+    assert m, "macro not found"
+    expr = m.group(1).replace("u", "")
+    assert re.fullmatch(r"[0-9* ]+", expr), expr
+    value = 1
+    for factor in expr.split("*"):
+        value *= int(factor)
+    assert value == binding.NOALLOC_MAX_SCRATCH_BYTES
+
+
 def test_every_declared_function_is_exported(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
@@ -85,9 +99,12 @@ def test_backward_rejects_bad_arguments_without_a_device(lib):
 
 
 def test_workspace_size_formula(lib):
-    # D and LSE2 (fp32) plus the fp32 dQ accumulator, rows padded to 128 per head
-    assert lib.fa_backward_workspace_bytes(2, 3, 200, 64) == 2 * 3 * 256 * (4 + 4 + 64 * 4)
-    assert lib.fa_backward_workspace_bytes(1, 1, 128, 128) == 128 * (8 + 512)
+    # D and LSE2 (fp32) plus the fp32 dQ accumulator, rows padded to 128 per
+    # head, then one int32 counter per 128-row query block padded to 256 bytes
+    assert lib.fa_backward_workspace_bytes(2, 3, 200, 64) == 2 * 3 * 256 * (4 + 4 + 64 * 4) + 256
+    assert lib.fa_backward_workspace_bytes(1, 1, 128, 128) == 128 * (8 + 512) + 256
+    assert lib.fa_backward_workspace_bytes(4, 16, 2048, 64) == (
+        4 * 16 * 2048 * (8 + 256) + 4 * 16 * 16 * 4)
     assert lib.fa_backward_workspace_bytes(1, 1, 0, 64) == 0
 
 
@@ -104,8 +121,8 @@ def test_package_exports_resolve():
 
 def test_extended_entry_points_reject_bad_arguments_without_a_device(lib):
     """The documented INVALID_ARG / UNSUPPORTED cases of the grouped, padded,
-    dropout, E4M3, no-alloc and self-test entry points, all returned before
-    any device is touched."""
+    dropout, E4M3, deterministic, no-alloc and self-test entry points, all
+    returned before any device is touched."""
     INV, UNS = binding.FA_ERR_INVALID_ARG, binding.FA_ERR_UNSUPPORTED
     a = [16] * 5  # aligned fake pointers: Q, K, V, O, LSE
 
@@ -130,6 +147,15 @@ def test_extended_entry_points_reject_bad_arguments_without_a_device(lib):
                                    None) == INV
     assert lib.fa_backward_dropout(*p10, 16, None, 1, 2, 2, 8, 64, 0.125, 0, 0.1, 1, 0,
                                    None) == INV
+    # deterministic backward: the same argument checks as the dropout backward
+    assert lib.fa_backward_deterministic(*p10, 1 << 30, None, 1, 2, 2, 8, 64, 0.125, 0, 1.0, 1,
+                                         0, None) == INV
+    assert lib.fa_backward_deterministic(*p10, 16, None, 1, 2, 2, 8, 64, 0.125, 0, 0.0, 1, 0,
+                                         None) == INV
+    assert lib.fa_backward_deterministic(*p10, 1 << 30, None, 1, 6, 4, 8, 64, 0.125, 0, 0.0, 1,
+                                         0, None) == INV
+    assert lib.fa_backward_deterministic(*p10, 1 << 30, None, 1, 2, 2, 8, 80, 0.125, 0, 0.0, 1,
+                                         0, None) == UNS
     # no-alloc backward: problems beyond its built-in array are UNSUPPORTED
     p9 = [16] * 9
     assert lib.fa_backward_noalloc(*p9, 64, 16, 4096, 128, 0.088, 1, None) == UNS
