@@ -53,6 +53,12 @@ def test_h16_n16384_d128_causal_x2_sampled():
     check_forward_sampled(w.B, w.H, w.N, w.d, w.causal, input_scale=w.input_scale, n_random=4)
 
 
+def test_b4_h16_n2048_d64_causal_sampled():
+    """The forward of the forward + backward workload, every CTA checked."""
+    w = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
+    check_forward_sampled(w.B, w.H, w.N, w.d, w.causal, n_random=4)
+
+
 def test_deterministic():
     x = inputs(2, 4, 1100, 128, seed=7)
     o1, l1 = gpu_forward(x, True, 1 / math.sqrt(128))

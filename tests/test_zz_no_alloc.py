@@ -7,7 +7,9 @@ Collected last on purpose (file name), so a run that stops at the first
 failure has already run every other test.  Checked against the regular
 fa_backward entry point on the same inputs, within the backward band the
 parity tests use, on two calls in a row with different shapes, so that what
-the first call leaves in the shared array cannot leak into the second.
+the first call leaves in the shared array cannot leak into the second; and
+once directly against the fp64 oracle, so that a fault shared by both entry
+points would not pass unseen.
 """
 import ctypes
 import math
@@ -15,9 +17,11 @@ import math
 import pytest
 import torch
 
+import oracle
 from io_aware_exact_31_b200 import binding
+from io_aware_exact_31_b200.workloads import bf16_bits
 
-from _parity import TOL_GRAD_REL, inputs
+from _parity import TOL_GRAD_REL, grad_rel_err, inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +61,25 @@ def test_noalloc_matches_fa_backward_on_two_calls(first, second):
             assert torch.isfinite(g.float()).all(), name
             e = _rel(g, r)
             assert e <= TOL_GRAD_REL, f"{name}: rel diff {e:.3e} vs fa_backward"
+
+
+def test_noalloc_matches_the_oracle():
+    lib = binding.load_library()
+    B, H, N, d, causal = 1, 2, 333, 64, True
+    x = inputs(B, H, N, d, seed=25, with_dO=True)
+    q, k, v, do = (x[n].cuda() for n in ("Q", "K", "V", "dO"))
+    scale = 1.0 / math.sqrt(d)
+    o, lse = binding.forward(q, k, v, causal=causal, scale=scale)
+    got = [torch.full_like(q, float("nan")) for _ in range(3)]
+    st = _noalloc(lib, q, k, v, o, do, lse, *got, causal, scale)
+    assert st == binding.FA_OK, binding.status_str(st)
+    st, site = binding.check_device_error()
+    assert st == binding.FA_OK, f"device error {site:#x}"
+    refs = oracle.attention_backward(*(bf16_bits(x[n]) for n in ("Q", "K", "V", "dO")), scale,
+                                     causal)
+    for name, g, r in zip(("dQ", "dK", "dV"), got, refs):
+        e = grad_rel_err(g, r)
+        assert e <= TOL_GRAD_REL, f"{name}: rel err {e:.3e} vs the oracle"
 
 
 def test_noalloc_rejects_problems_beyond_its_array():
