@@ -177,7 +177,9 @@ def weak_scaling_tflops(flops_per_rank: float, world: int, ms_per_step_slowest: 
 
 
 def time_region(fn, steps, stream, sync):
-    """CUDA-event time of `steps` calls on `stream`, bracketed by sync()."""
+    """CUDA-event time of `steps` calls on `stream`, bracketed by sync().  The
+    host waits for the end event by polling with short sleeps, so that the
+    clock-sampling thread gets the interpreter while the GPU works."""
     import torch
     sync()
     start = torch.cuda.Event(enable_timing=True)
@@ -186,6 +188,8 @@ def time_region(fn, steps, stream, sync):
     for _ in range(steps):
         fn()
     end.record(stream)
+    while not end.query():
+        time.sleep(20e-6)
     end.synchronize()
     sync()
     return start.elapsed_time(end)  # ms
@@ -222,6 +226,23 @@ def run_gpu(args):
     if args.only == "fwd" and args.workload:
         w = WORKLOADS[args.workload]
 
+    fp8_cache = {}
+
+    def fp8_args(a):
+        """fa_forward_fp8 arguments for the bf16 buffers of `a`, quantised once."""
+        if id(a) not in fp8_cache:
+            ts, ds = [], []
+            for ptr_t in fwd_tensors[id(a)][:3]:
+                s_ = float(ptr_t.float().abs().max()) / 448.0
+                ts.append((ptr_t.float() / s_).to(torch.float8_e4m3fn))
+                ds.append(s_)
+            fp8_cache[id(a)] = (ts, ds)
+        (q8_, k8_, v8_), ds = fp8_cache[id(a)]
+        return (q8_.data_ptr(), k8_.data_ptr(), v8_.data_ptr(), a[3], a[4], *ds, w.B, w.H, w.H,
+                w.N, w.d, w.scale, int(w.causal), binding.ctypes.c_void_p(a[-1]))
+
+    fwd_tensors = {}
+
     def fwd_setup(w):
         x = workload_inputs(w, seed=rank)
         q, k, v = (x[n].cuda() for n in ("Q", "K", "V"))
@@ -229,12 +250,20 @@ def run_gpu(args):
         lse = torch.empty(w.B, w.H, w.N, device="cuda", dtype=torch.float32)
         args_ = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B,
                  w.H, w.N, w.d, w.scale, int(w.causal), sh)
+        fwd_tensors[id(args_)] = (q, k, v)
         return x, (q, k, v, o, lse), args_
 
     def launch_fwd(a):
         st = lib.fa_forward(*a[:-1], binding.ctypes.c_void_p(a[-1]))
         if st != 0:
             raise binding.FaError(st, "fa_forward")
+
+    if args.only == "fwd" and args.fp8:
+        # profiler runs of the E4M3 forward: the workload quantised per tensor
+        def launch_fwd(a):  # noqa: F811
+            st = lib.fa_forward_fp8(*fp8_args(a))
+            if st != 0:
+                raise binding.FaError(st, "fa_forward_fp8")
 
     if args.only == "fwd" and args.dropout > 0:
         # profiler runs of the dropout forward: same workload, fa_forward_dropout
@@ -438,11 +467,17 @@ def run_gpu(args):
         binding.forward(q5, k5, v5, causal=True, scale=w5.scale, out=o5, lse=l5,
                         dropout_p=DROPOUT_P, seed=99, offset=0)
 
+    def bwd_det_step():
+        binding.backward(q5, k5, v5, o5, do5, l5, causal=True, scale=w5.scale, dq=dq5, dk=dk5,
+                         dv=dv5, workspace=ws, deterministic=True)
+
     for _ in range(args.warmup):
         bwd_step()
         fwd5_step()
+        bwd_det_step()
     msb = max_ranks(time_region(bwd_step, args.steps, stream, barrier)) / args.steps
     msf = max_ranks(time_region(fwd5_step, args.steps, stream, barrier)) / args.steps
+    msbdet = max_ranks(time_region(bwd_det_step, args.steps, stream, barrier)) / args.steps
     for _ in range(args.warmup):
         fwd5_drop_step()
         bwd5_drop_step()
@@ -455,6 +490,11 @@ def run_gpu(args):
                       "fwd_tflops": round(w5.fwd_flops / (msf * 1e-3) / 1e12, 1),
                       "bwd_tflops": round(w5.bwd_flops / (msb * 1e-3) / 1e12, 1),
                       "bwd_launches_per_step": 3,
+                      "deterministic_bwd": {
+                          "ms": round(msbdet, 4),
+                          "tflops": round(w5.bwd_flops / (msbdet * 1e-3) / 1e12, 1),
+                          "cost_vs_default": round(msbdet / msb - 1.0, 4),
+                          "how": "dQ blocks added in ascending key-block order"},
                       "dropout": {"p": DROPOUT_P, "fwd_ms": round(msfd, 4),
                                   "bwd_ms": round(msbd, 4),
                                   "fwd_tflops": round(w5.fwd_flops / (msfd * 1e-3) / 1e12, 1),
@@ -716,8 +756,12 @@ def torch_sdpa_context(torch, w, w5, stream, args, max_ranks):
 
 
 def run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank):
-    """Backward of the 4x16x2048x64 causal workload alone (for profiler runs)."""
+    """Backward of the 4x16x2048x64 causal workload alone (for profiler runs);
+    --bwd-d 128 takes the same shape at head dimension 128."""
+    import dataclasses
     w5 = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
+    if args.bwd_d != w5.d:
+        w5 = dataclasses.replace(w5, name=f"b4_h16_n2048_d{args.bwd_d}_causal_bwd", d=args.bwd_d)
     x5 = workload_inputs(w5, seed=rank)
     q, k, v, do = (x5[n].cuda() for n in ("Q", "K", "V", "dO"))
     o, lse = binding.forward(q, k, v, causal=True, scale=w5.scale)
@@ -731,7 +775,7 @@ def run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank):
 
     def step():
         binding.backward(q, k, v, o, do, lse, causal=True, scale=w5.scale, dq=dq, dk=dk, dv=dv,
-                         workspace=ws, dropout_p=p, seed=99)
+                         workspace=ws, dropout_p=p, seed=99, deterministic=args.deterministic)
 
     for _ in range(args.warmup):
         step()
@@ -739,7 +783,8 @@ def run_bwd_only(args, torch, binding, WORKLOADS, workload_inputs, rank):
     ms = time_region(step, args.steps, stream, torch.cuda.synchronize) / args.steps
     return {"metric": METRIC, "value": round(w5.bwd_flops / (ms * 1e-3) / 1e12, 1),
             "unit": UNIT, "ms_per_step": round(ms, 4), "steps": args.steps,
-            "config": {"workload": f"{w5.name} bwd", "dropout_p": p},
+            "config": {"workload": f"{w5.name} bwd", "dropout_p": p,
+                       "deterministic": args.deterministic},
             "gpu_launches": 3 * args.steps}
 
 
@@ -917,6 +962,12 @@ def main():
                     help="time only the headline forward / the backward (profiler runs)")
     ap.add_argument("--workload", default=None,
                     help="workload name of the --only fwd run (default: the headline)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="--only fwd: time the E4M3 forward of the workload (d = 128)")
+    ap.add_argument("--bwd-d", type=int, default=64, choices=[64, 128],
+                    help="--only bwd: head dimension of the 4x16x2048 causal backward")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="--only bwd: the deterministic backward")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="attention-dropout rate of the --only fwd / --only bwd runs")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
