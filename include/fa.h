@@ -94,18 +94,18 @@ fa_status fa_forward_varlen(const void *Q, const void *K, const void *V, void *O
  * on the normalised probabilities:
  *     O_i = sum_j P_ij z_ij / q v_j,   LSE as without dropout
  * with the keep bit z_ij of query i, key j of query head bh = b * H + h taken
- * from the counter-based generator Philox-4x32-10 (Salmon et al., "Parallel
- * Random Numbers: As Easy as 1, 2, 3", SC'11):
- *     W = Philox(counter = (j / 8, i, bh, offset), key = (seed & 0xffffffff, seed >> 32))
- *     u = (W[(j % 8) / 2] >> (16 * (j % 2))) & 0x7fff        (15-bit uniform)
- *     z_ij = (u < t),  t = floor((1 - dropout_p) * 2^15 + 1/2),  q = t / 2^15
+ * from the counter-based generator Philox-4x32 with 7 rounds (Salmon et al.,
+ * "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11):
+ *     W = Philox(counter = (j / 16, i, bh, offset), key = (seed & 0xffffffff, seed >> 32))
+ *     u = (W[(j % 16) / 4] >> (8 * (2 * (j % 2) + (j % 4) / 2))) & 0xff   (8-bit uniform)
+ *     z_ij = (u < t),  t = floor((1 - dropout_p) * 2^8 + 1/2),  q = t / 2^8
  * (i, j counted from the start of the sequence).  q, the keep probability, is
- * the multiple of 2^-15 nearest to 1 - dropout_p, and dividing by it keeps
+ * the multiple of 2^-8 nearest to 1 - dropout_p, and dividing by it keeps
  * the output unbiased.  The same (seed, offset) given to fa_backward_dropout
  * regenerates the mask; a caller that needs a fresh mask per call changes
  * either.
- *   dropout_p : in [0, 1 - 2^-16] (FA_ERR_INVALID_ARG otherwise, NaN
- *               included); values below 2^-16 (t = 2^15) are exactly
+ *   dropout_p : in [0, 1 - 2^-9] (FA_ERR_INVALID_ARG otherwise, NaN
+ *               included); values below 2^-9 (t = 2^8) are exactly
  *               fa_forward_varlen.
  * Other arguments as fa_forward_varlen (seqlens may be NULL; K/V with H_kv
  * heads).  The keep-bit generation costs integer work in the softmax warps.

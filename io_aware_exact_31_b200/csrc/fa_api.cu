@@ -86,25 +86,25 @@ fa_status check_heads(int H, int Hkv) {
 }
 
 // Attention-dropout parameters from (p, seed, offset): keep threshold
-// t = floor((1 - p) 2^15 + 1/2) on 15-bit uniforms, keep scale 2^15 / t, and
-// the ten Philox round keys.  *on = false when t = 2^15 (p < 2^-16: nothing is
-// ever dropped), which runs the kernels without dropout; t = 0 is rejected.
+// t = floor((1 - p) 2^8 + 1/2) on 8-bit uniforms, keep scale 2^8 / t, and the
+// Philox round keys.  *on = false when t = 2^8 (p < 2^-9: nothing is ever
+// dropped), which runs the kernels without dropout; t = 0 is rejected.
 fa_status make_dropout(float p, uint64_t seed, uint32_t offset, DropoutParams* d, bool* on) {
     if (!(p >= 0.f && p < 1.f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
-    const double t = std::floor((1.0 - static_cast<double>(p)) * 32768.0 + 0.5);
+    const double t = std::floor((1.0 - static_cast<double>(p)) * 256.0 + 0.5);
     if (t < 1.0) return FA_ERR_INVALID_ARG;
-    *on = t < 32768.0;
+    *on = t < 256.0;
     uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
-    for (int r = 0; r < 10; ++r) {
+    for (int r = 0; r < PHILOX_ROUNDS; ++r) {
         d->key[2 * r] = k0;
         d->key[2 * r + 1] = k1;
         k0 += 0x9E3779B9u;  // Weyl increments of Philox-4x32
         k1 += 0xBB67AE85u;
     }
     d->offset = offset;
-    const uint32_t ref = (static_cast<uint32_t>(t) - 1u) | 0x8000u;
+    const uint32_t ref = 0x8000u + static_cast<uint32_t>(t) - 1u;
     d->lanes_ref = ref | (ref << 16);
-    d->keep_scale = static_cast<float>(32768.0 / t);
+    d->keep_scale = static_cast<float>(256.0 / t);
     return FA_OK;
 }
 

@@ -520,10 +520,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                         if constexpr (DROP) {
                             // Dropped weights leave the P.V product but stay in
                             // both row sums (the softmax is of undropped scores).
-                            // keys 64h + 2i (low half) and 64h + 2i + 1 (high half)
-                            const int o = (2 * i) % 32;
-                            const uint32_t kb =
-                                (keep[(h * 64 + 2 * i) / 32] >> (4 * (o / 8) + (o % 8) / 2)) & 0x00010001u;
+                            // keys 64h + 2i (low half) and 64h + 2i + 1 (high half):
+                            // key pair 32h + i of keep_bits_row128's layout
+                            const uint32_t kb = (keep[2 * h + i / 16] >> (i % 16)) & 0x00010001u;
                             pk[i] &= kb * 0xFFFFu;
                         }
                     }

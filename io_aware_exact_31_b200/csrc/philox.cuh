@@ -8,38 +8,43 @@
 // scores.
 //
 // The keep bit z_ij of query i, key j of query head bh = b * H + h comes from
-// the counter-based generator Philox-4x32-10 (Salmon, Moraes, Dror, Shaw,
-// "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11):
-//     W = Philox(counter = (j / 8, i, bh, offset), key = (seed lo, seed hi))
-//     u = (W[(j % 8) / 2] >> 16 (j % 2)) & 0x7FFF            (15-bit uniform)
-//     z_ij = u < t,  t = floor((1 - p) 2^15 + 1/2),  q = t / 2^15
-// so one call serves eight consecutive keys of a row (two per 32-bit word,
-// one per 16-bit half), and the backward pass regenerates exactly the
-// forward's mask from (seed, offset).  With 15-bit numbers in 16-bit lanes
-// both halves of a word are compared with one borrow-free subtraction.
+// the counter-based generator Philox-4x32 (Salmon, Moraes, Dror, Shaw,
+// "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) run for 7 rounds (the
+// paper reports Philox-4x32 passing TestU01's Crush batteries from 7 rounds
+// on; its default of 10 adds a safety margin):
+//     W = Philox(counter = (j / 16, i, bh, offset), key = (seed lo, seed hi))
+//     u = byte 2 (j % 2) + (j % 4) / 2 of W[(j % 16) / 4]        (8-bit uniform)
+//     z_ij = u < t,  t = floor((1 - p) 2^8 + 1/2),  q = t / 2^8
+// so one call serves sixteen consecutive keys of a row, and the backward pass
+// regenerates exactly the forward's mask from (seed, offset).  The byte order
+// (keys 4w, 4w+1, 4w+2, 4w+3 in bytes 0, 2, 1, 3 of word w) puts a pair of
+// keys 2c, 2c + 1 in the low bytes of the two 16-bit halves of a word, so one
+// borrow-free subtraction decides both (keep_lanes).
 #pragma once
 
 #include <stdint.h>
 
 namespace fa {
 
+constexpr int PHILOX_ROUNDS = 7;
+
 struct DropoutParams {
-    uint32_t key[20];     // Philox round keys: (k0, k1) + r (W0, W1), r = 0..9
-    uint32_t offset;      // counter word 3
-    uint32_t lanes_ref;   // ((t - 1) | 0x8000) in both 16-bit halves
-    float keep_scale;     // 2^15 / t = 1 / q
+    uint32_t key[2 * PHILOX_ROUNDS];  // round keys: (k0, k1) + r (W0, W1), r = 0..6
+    uint32_t offset;                  // counter word 3
+    uint32_t lanes_ref;               // (0x8000 + t - 1) in both 16-bit halves
+    float keep_scale;                 // 2^8 / t = 1 / q
 };
 
-// Philox-4x32 with ten rounds, as the SC'11 paper defines it: each round takes
-// the 64-bit products of counter words 0 and 2 with the multipliers M0, M1 and
-// forms (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)); the
-// key of round r is the seed plus r times the Weyl increments (precomputed on
-// the host into DropoutParams::key).
-__device__ __forceinline__ uint4 philox4x32_10(const DropoutParams& d, uint32_t c0, uint32_t c1,
-                                               uint32_t c2, uint32_t c3) {
+// Philox-4x32 as the SC'11 paper defines it, PHILOX_ROUNDS rounds: each round
+// takes the 64-bit products of counter words 0 and 2 with the multipliers
+// M0, M1 and forms (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1,
+// lo(M0 c0)); the key of round r is the seed plus r times the Weyl
+// increments (precomputed on the host into DropoutParams::key).
+__device__ __forceinline__ uint4 philox4x32(const DropoutParams& d, uint32_t c0, uint32_t c1,
+                                            uint32_t c2, uint32_t c3) {
     constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
 #pragma unroll
-    for (int r = 0; r < 10; ++r) {
+    for (int r = 0; r < PHILOX_ROUNDS; ++r) {
         const unsigned long long p0 = static_cast<unsigned long long>(M0) * c0;
         const unsigned long long p1 = static_cast<unsigned long long>(M1) * c2;
         const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ d.key[2 * r];
@@ -52,77 +57,83 @@ __device__ __forceinline__ uint4 philox4x32_10(const DropoutParams& d, uint32_t 
     return make_uint4(c0, c1, c2, c3);
 }
 
-// Keep decisions of both 16-bit halves of one output word: bit 15 is set iff
-// the low half keeps its key, bit 31 iff the high half does.  In each lane
-// (0x8000 + t - 1) - u lies in [1, 0xFFFE] for u, t - 1 < 2^15, so no borrow
-// crosses lanes, and its bit 15 is set iff u <= t - 1.
-__device__ __forceinline__ uint32_t keep_pair_bits(uint32_t w, uint32_t lanes_ref) {
-    return (lanes_ref - (w & 0x7FFF7FFFu)) & 0x80008000u;
+// Keep decisions of the two keys whose 8-bit numbers sit in the low bytes of
+// the 16-bit halves of v (the high bytes zero): bit 15 is set iff the low half
+// keeps its key, bit 31 iff the high half does.  In each lane
+// (0x8000 + t - 1) - u lies in [0x7F01, 0x80FF] for u, t - 1 < 2^8, so no
+// borrow crosses lanes, and its bit 15 is set iff u <= t - 1.
+__device__ __forceinline__ uint32_t keep_lanes(uint32_t v, uint32_t lanes_ref) {
+    return (lanes_ref - v) & 0x80008000u;
+}
+
+// The decisions of the 16 keys of one call as two bits per key pair: pair
+// 2w + s (keys 8w.. of the word order above: s = 0 the bytes 0/2, s = 1 the
+// bytes 1/3 of word w) at bits x and x + 16, x = 2 w + s, the low key (even)
+// in the low half.
+__device__ __forceinline__ uint32_t keep_bits16(const uint4 w, uint32_t lanes_ref) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    uint32_t b = 0;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        b |= (keep_lanes(ww[x] & 0x00FF00FFu, lanes_ref) >> 15) << (2 * x);
+        b |= (keep_lanes((ww[x] >> 8) & 0x00FF00FFu, lanes_ref) >> 15) << (2 * x + 1);
+    }
+    return b;
 }
 
 // Keep bits of query i for the 128 keys [j0, j0 + 128) (j0 a multiple of
-// 128): bit 16 e + 4 k + x of keep[c] for key j0 + 32 c + 8 k + 2 x + e.
+// 128): keys 2P (bit P % 16) and 2P + 1 (bit 16 + P % 16) of keep[P / 16],
+// for the key pairs P = 0..63 of the block.
 __device__ __forceinline__ void keep_bits_row128(const DropoutParams& d, uint32_t j0, uint32_t i,
                                                  uint32_t bh, uint32_t (&keep)[4]) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) keep[c] = 0;
-#pragma unroll 1
-    for (int k = 0; k < 4; ++k) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint4 w = philox4x32_10(d, (j0 >> 3) + 4 * c + k, i, bh, d.offset);
-            const uint32_t b = (keep_pair_bits(w.x, d.lanes_ref) >> 15) |
-                               (keep_pair_bits(w.y, d.lanes_ref) >> 14) |
-                               (keep_pair_bits(w.z, d.lanes_ref) >> 13) |
-                               (keep_pair_bits(w.w, d.lanes_ref) >> 12);
-            keep[c] |= b << (4 * k);
-        }
+    for (int c = 0; c < 4; ++c) {
+        const uint32_t lo = keep_bits16(philox4x32(d, (j0 >> 4) + 2 * c, i, bh, d.offset),
+                                        d.lanes_ref);
+        const uint32_t hi = keep_bits16(philox4x32(d, (j0 >> 4) + 2 * c + 1, i, bh, d.offset),
+                                        d.lanes_ref);
+        // a call covers 8 pairs: bits 0..7 (low keys) and 16..23 (high keys)
+        keep[c] = (lo & 0x00FF00FFu) | ((hi & 0x00FF00FFu) << 8);
     }
-}
-
-// Spread the 8 low bits of x eight apart: bit m goes to bit 8m.
-__device__ __forceinline__ unsigned long long spread8(uint32_t x) {
-    unsigned long long v = x & 0xFFu;
-    v = (v | (v << 28)) & 0x0000000F0000000Full;
-    v = (v | (v << 14)) & 0x0003000300030003ull;
-    v = (v | (v << 7)) & 0x0101010101010101ull;
-    return v;
 }
 
 // Keep bits of one key (this lane's) against 64 consecutive queries q0 .. q0+63,
-// bit c for query q0 + c, with the eight lanes of an aligned lane octet
-// holding the eight keys of one Philox group (key & 7 == lane & 7).  Each lane
-// makes the 8 calls for the queries q0 + 8m + (lane & 7) -- every call yields
-// the decisions of all eight keys of the group -- and the octet exchanges them
-// with seven xor shuffles (an 8 x 8 transpose of bytes).
+// bit c for query q0 + c, with the sixteen lanes of an aligned half-warp
+// holding the sixteen keys of one Philox group (key & 15 == lane & 15).  Each
+// lane makes the 4 calls for the queries q0 + 16 m + (lane & 15) -- every call
+// yields the decisions of all sixteen keys of the group -- and the half-warp
+// exchanges them with fifteen xor shuffles (a 16 x 16 bit transpose per m).
 __device__ __forceinline__ unsigned long long keep_bits_key_row(const DropoutParams& d, uint32_t key,
                                                                 uint32_t q0, uint32_t bh,
                                                                 uint32_t lane) {
-    const uint32_t w = lane & 7u;
-    // a[x] bit m (low half) and bit 16 + m (high half): keys 2x and 2x + 1 of
-    // the group against query q0 + 8m + w.
-    uint32_t a[4] = {0u, 0u, 0u, 0u};
-#pragma unroll 2
-    for (uint32_t m = 0; m < 8; ++m) {
-        const uint4 v = philox4x32_10(d, key >> 3, q0 + 8 * m + w, bh, d.offset);
-        a[0] |= keep_pair_bits(v.x, d.lanes_ref) >> (15 - m);
-        a[1] |= keep_pair_bits(v.y, d.lanes_ref) >> (15 - m);
-        a[2] |= keep_pair_bits(v.z, d.lanes_ref) >> (15 - m);
-        a[3] |= keep_pair_bits(v.w, d.lanes_ref) >> (15 - m);
-    }
-    // Decisions of key x of the group (8 bits, bit m), x = 0..7.
-    auto pick = [&](uint32_t x) {
-        const uint32_t hi2 = x >> 1;
-        const uint32_t r = (hi2 == 0) ? a[0] : (hi2 == 1) ? a[1] : (hi2 == 2) ? a[2] : a[3];
-        return (r >> (16 * (x & 1u))) & 0xFFu;
-    };
-    unsigned long long M = spread8(pick(w)) << w;
+    const uint32_t w = lane & 15u;
+    // D bit 16 m + k: key k of the group (k = 0..15) against query q0 + 16 m + w.
+    unsigned long long D = 0ull;
 #pragma unroll
-    for (uint32_t k = 1; k < 8; ++k) {
-        // The partner lane ^ k sends its decisions for key w (= its (lane & 7) ^ k);
-        // they cover the queries q0 + 8m + (w ^ k).
-        const uint32_t got = __shfl_xor_sync(0xffffffffu, pick(w ^ k), k);
-        M |= spread8(got) << (w ^ k);
+    for (uint32_t m = 0; m < 4; ++m) {
+        const uint32_t b = keep_bits16(philox4x32(d, key >> 4, q0 + 16 * m + w, bh, d.offset),
+                                       d.lanes_ref);
+        // b: pair x = k / 2 at bit x (even key) and bit 16 + x (odd key)
+        uint32_t byk = 0;  // bit k = key k
+#pragma unroll
+        for (int x = 0; x < 8; ++x) byk |= ((b >> x) & 1u) << (2 * x) | ((b >> (16 + x)) & 1u) << (2 * x + 1);
+        D |= static_cast<unsigned long long>(byk) << (16 * m);
+    }
+    constexpr unsigned long long EVERY16 = 0x0001000100010001ull;
+    // Own decisions: key w against queries q0 + 16 m + w.
+    unsigned long long M = ((D >> w) & EVERY16) << w;
+#pragma unroll
+    for (uint32_t k = 1; k < 16; ++k) {
+        // Send the partner (lane ^ k) its key's decisions (key w ^ k) for the
+        // queries q0 + 16 m + w, packed into 4 bits; receive this key's
+        // decisions for the queries q0 + 16 m + (w ^ k).
+        const unsigned long long s = (D >> (w ^ k)) & EVERY16;
+        const uint32_t packed = static_cast<uint32_t>(s | (s >> 15) | (s >> 30) | (s >> 45)) & 0xFu;
+        const uint32_t got = __shfl_xor_sync(0xffffffffu, packed, k);
+        const unsigned long long g = (got & 1u) | (static_cast<unsigned long long>((got >> 1) & 1u) << 16) |
+                                     (static_cast<unsigned long long>((got >> 2) & 1u) << 32) |
+                                     (static_cast<unsigned long long>((got >> 3) & 1u) << 48);
+        M |= g << (w ^ k);
     }
     return M;
 }

@@ -71,6 +71,8 @@ def load(path: str | None = None):
                                                             vp, vp, vp]
     lib.oracle_philox4x32_10.argtypes = [vp, vp, vp]
     lib.oracle_philox4x32_10.restype = None
+    lib.oracle_philox4x32_7.argtypes = [vp, vp, vp]
+    lib.oracle_philox4x32_7.restype = None
     lib.oracle_dropout_keep_mask.argtypes = [i64, i64, i64, dbl, u64, u32, vp]
     lib.oracle_softmax_partial.argtypes = [vp, i64, vp, i64, vp, vp, vp]
     lib.oracle_softmax_merge.argtypes = [dbl, dbl, vp, dbl, dbl, vp, i64, vp, vp, vp]
@@ -316,15 +318,23 @@ def attention_backward_dropout_heads(Q, K, V, dO, scale: float, causal: bool, p_
     return dQ, dK, dV
 
 
-def philox4x32_10(counter, key, lib=None):
-    """The four 32-bit output words of Philox-4x32-10 for a 4-word counter and 2-word key."""
-    lib = lib or load()
+def _philox(fn, counter, key):
     c = np.ascontiguousarray(counter, dtype=np.uint32)
     k = np.ascontiguousarray(key, dtype=np.uint32)
     assert c.shape == (4,) and k.shape == (2,)
     out = np.empty(4, np.uint32)
-    lib.oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    fn(_ptr(c), _ptr(k), _ptr(out))
     return out
+
+
+def philox4x32_10(counter, key, lib=None):
+    """The four 32-bit output words of Philox-4x32-10 for a 4-word counter and 2-word key."""
+    return _philox((lib or load()).oracle_philox4x32_10, counter, key)
+
+
+def philox4x32_7(counter, key, lib=None):
+    """Philox-4x32 with 7 rounds (the dropout generator)."""
+    return _philox((lib or load()).oracle_philox4x32_7, counter, key)
 
 
 def dropout_keep_mask(B: int, H: int, N: int, p_drop: float, seed: int, offset: int = 0,

@@ -54,21 +54,24 @@
  *           probabilities, O_i = sum_j P_ij z_ij / (1 - p) v_j with z_ij in
  *           {0, 1} kept with probability 1 - p; LSE is that of the undropped
  *           scores.  The page gives no random-number convention either:
- *           z_ij comes from the counter-based generator Philox-4x32-10
- *           (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as
- *           1, 2, 3", SC'11), called with
- *             counter = (j / 8, i, b * H + h, offset), key = (seed mod 2^32,
+ *           z_ij comes from the counter-based generator Philox-4x32 (Salmon,
+ *           Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3",
+ *           SC'11) with 7 rounds (the paper reports Philox-4x32 passing
+ *           TestU01's Crush batteries from 7 rounds on; its default of 10
+ *           adds a safety margin), called with
+ *             counter = (j / 16, i, b * H + h, offset), key = (seed mod 2^32,
  *                       seed / 2^32)
  *           for query i, key j of query head h of batch b (positions counted
- *           from the start of the sequence).  Each 32-bit output word holds
- *           two 15-bit numbers, u = (word >> 16 e) mod 2^15 for e = 0, 1;
- *           key j takes word (j mod 8) / 2, half e = j mod 2, and is kept iff
- *           u < t = floor((1 - p) 2^15 + 1/2).  The keep probability is then
- *           q = t / 2^15 (the nearest multiple of 2^-15 to 1 - p) and kept
+ *           from the start of the sequence).  One call gives the 8-bit
+ *           numbers of 16 consecutive keys: key j takes word (j mod 16) / 4,
+ *           byte 2 (j mod 2) + (j mod 4) / 2 of it (keys 4w, 4w+1, 4w+2,
+ *           4w+3 in bytes 0, 2, 1, 3 of word w), and is kept iff
+ *           u < t = floor((1 - p) 2^8 + 1/2).  The keep probability is then
+ *           q = t / 2^8 (the nearest multiple of 2^-8 to 1 - p) and kept
  *           weights are scaled by 1 / q, so the dropout stays unbiased:
  *             O_i = sum_j P_ij z_ij / q v_j.
- *           t = 2^15 (p < 2^-16) keeps everything; p > 1 - 2^-16 (t = 0)
- *           is rejected.
+ *           t = 2^8 (p < 2^-9) keeps everything; p > 1 - 2^-9 (t = 0) is
+ *           rejected.
  *
  * Every function returns 0 on success, -1 on a bad argument, -2 if memory
  * could not be allocated.
@@ -118,19 +121,19 @@ static int bad_seqlens(const int32_t *seqlens, int64_t B, int64_t N)
 }
 
 /*
- * [DROP] Philox-4x32 with 10 rounds, as the SC'11 paper defines it: each
+ * [DROP] Philox-4x32 with R rounds, as the SC'11 paper defines it: each
  * round multiplies counter words 0 and 2 by the constants M0, M1 into 64-bit
  * products (hi, lo), and the new counter is
  *     (hi(M1 c2) ^ c1 ^ k0,  lo(M1 c2),  hi(M0 c0) ^ c3 ^ k1,  lo(M0 c0));
  * between rounds the key is bumped by the Weyl constants W0, W1.
  */
-void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+static void philox4x32(const uint32_t ctr[4], const uint32_t key[2], int rounds, uint32_t out[4])
 {
     const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
     const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
     uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
     uint32_t k0 = key[0], k1 = key[1];
-    for (int r = 0; r < 10; ++r) {
+    for (int r = 0; r < rounds; ++r) {
         const uint64_t p0 = (uint64_t)M0 * c0, p1 = (uint64_t)M1 * c2;
         const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
         const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
@@ -147,20 +150,33 @@ void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t
     out[3] = c3;
 }
 
+/* The paper's default, 10 rounds (the form its known-answer vectors cover). */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    philox4x32(ctr, key, 10, out);
+}
+
+/* The [DROP] generator: 7 rounds. */
+#define DROP_ROUNDS 7
+void oracle_philox4x32_7(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    philox4x32(ctr, key, DROP_ROUNDS, out);
+}
+
 /* [DROP] parameters; NULL or p == 0 means no dropout. */
 struct dropout {
     double p;            /* requested probability of dropping, [0, 1) */
     uint32_t key[2];     /* the seed */
     uint32_t offset;     /* counter word 3 */
-    uint32_t threshold;  /* t = floor((1 - p) 2^15 + 1/2): keep iff u < t */
-    double keep_scale;   /* 2^15 / t = 1 / (keep probability) */
+    uint32_t threshold;  /* t = floor((1 - p) 2^8 + 1/2): keep iff u < t */
+    double keep_scale;   /* 2^8 / t = 1 / (keep probability) */
 };
 
 static int make_dropout(struct dropout *dr, double p, uint64_t seed, uint32_t offset)
 {
     if (!(p >= 0.0 && p < 1.0))
         return -1;
-    const double t = floor((1.0 - p) * 32768.0 + 0.5);
+    const double t = floor((1.0 - p) * 256.0 + 0.5);
     if (t < 1.0)
         return -1;
     dr->p = p;
@@ -168,17 +184,17 @@ static int make_dropout(struct dropout *dr, double p, uint64_t seed, uint32_t of
     dr->key[1] = (uint32_t)(seed >> 32);
     dr->offset = offset;
     dr->threshold = (uint32_t)t;
-    dr->keep_scale = 32768.0 / t;
+    dr->keep_scale = 256.0 / t;
     return 0;
 }
 
 /* z_ij of [DROP] for query i, key j of query head bh = b * H + h. */
 static int dropout_keep(const struct dropout *dr, int64_t bh, int64_t i, int64_t j)
 {
-    const uint32_t ctr[4] = {(uint32_t)(j / 8), (uint32_t)i, (uint32_t)bh, dr->offset};
+    const uint32_t ctr[4] = {(uint32_t)(j / 16), (uint32_t)i, (uint32_t)bh, dr->offset};
     uint32_t w[4];
-    oracle_philox4x32_10(ctr, dr->key, w);
-    const uint32_t u = (w[(j % 8) / 2] >> (16 * (j % 2))) & 0x7FFFu;
+    philox4x32(ctr, dr->key, DROP_ROUNDS, w);
+    const uint32_t u = (w[(j % 16) / 4] >> (8 * (2 * (j % 2) + (j % 4) / 2))) & 0xFFu;
     return u < dr->threshold;
 }
 
