@@ -405,13 +405,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         const int nt = n_tile[t];
         const int tile_first_q = q0 + t * FWD_BM;
         for (int j = 0; j < nt; ++j) {
-            // Dropout keep bits of this row for keys [128 j, 128 j + 128)
-            // (layout of keep_bits_row128).  They depend only on the indices,
-            // so they are made while S_t(j) is still on the tensor core.
-            uint32_t keep[4] = {~0u, ~0u, ~0u, ~0u};
-            if constexpr (DROP)
-                keep_bits_row128(p.drop, static_cast<uint32_t>(j * FWD_BN), static_cast<uint32_t>(q),
-                                 static_cast<uint32_t>(bh), keep);
+            uint4 dw = make_uint4(0u, 0u, 0u, 0u);  // DROP: Philox output of the current 16 keys
             if (!(ok = mbar_wait_warp(&bars->s_full[t], j & 1, g, 9 + t))) break;
             tc_fence_after();
             uint32_t sr[128];
@@ -520,10 +514,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                         if constexpr (DROP) {
                             // Dropped weights leave the P.V product but stay in
                             // both row sums (the softmax is of undropped scores).
-                            // keys 64h + 2i (low half) and 64h + 2i + 1 (high half):
-                            // key pair 32h + i of keep_bits_row128's layout
-                            const uint32_t kb = (keep[2 * h + i / 16] >> (i % 16)) & 0x00010001u;
-                            pk[i] &= kb * 0xFFFFu;
+                            // Keys 64h + 2i (low half of pk[i]) and 64h + 2i + 1
+                            // (high half): one Philox call per 16 keys, made here
+                            // where its integer work overlaps the exponentials;
+                            // the pair's bytes sit in the two 16-bit lanes of
+                            // word (i % 8) / 2 (bytes 0/2 for even i, 1/3 for odd
+                            // i), and keep_lanes turns each lane's decision into
+                            // bit 15 / bit 31, spread here to a 16-bit mask.
+                            if (i % 8 == 0)
+                                dw = philox4x32(p.drop,
+                                                static_cast<uint32_t>((j * FWD_BN) / 16 + 4 * h + i / 8),
+                                                static_cast<uint32_t>(q), static_cast<uint32_t>(bh),
+                                                p.drop.offset);
+                            const uint32_t wd = ((i % 8) / 2 == 0)   ? dw.x
+                                                : ((i % 8) / 2 == 1) ? dw.y
+                                                : ((i % 8) / 2 == 2) ? dw.z
+                                                                     : dw.w;
+                            const uint32_t lanes =
+                                (i % 2 == 0) ? (wd & 0x00FF00FFu) : ((wd >> 8) & 0x00FF00FFu);
+                            pk[i] &= (keep_lanes(lanes, p.drop.lanes_ref) >> 15) * 0xFFFFu;
                         }
                     }
                 }

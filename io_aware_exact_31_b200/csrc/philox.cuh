@@ -66,35 +66,20 @@ __device__ __forceinline__ uint32_t keep_lanes(uint32_t v, uint32_t lanes_ref) {
     return (lanes_ref - v) & 0x80008000u;
 }
 
-// The decisions of the 16 keys of one call as two bits per key pair: pair
-// 2w + s (keys 8w.. of the word order above: s = 0 the bytes 0/2, s = 1 the
-// bytes 1/3 of word w) at bits x and x + 16, x = 2 w + s, the low key (even)
-// in the low half.
+// The decisions of the 16 keys of one call, bit k for key k: in word w the
+// even lanes (bytes 0, 2) hold keys 4w, 4w + 1 and the odd lanes (bytes 1, 3)
+// keys 4w + 2, 4w + 3.  (The forward applies keep_lanes to the words directly,
+// in its exponential loop.)
 __device__ __forceinline__ uint32_t keep_bits16(const uint4 w, uint32_t lanes_ref) {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
     uint32_t b = 0;
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
-        b |= (keep_lanes(ww[x] & 0x00FF00FFu, lanes_ref) >> 15) << (2 * x);
-        b |= (keep_lanes((ww[x] >> 8) & 0x00FF00FFu, lanes_ref) >> 15) << (2 * x + 1);
+        const uint32_t e = keep_lanes(ww[x] & 0x00FF00FFu, lanes_ref);
+        const uint32_t o = keep_lanes((ww[x] >> 8) & 0x00FF00FFu, lanes_ref);
+        b |= (((e >> 15) & 1u) | ((e >> 30) & 2u) | ((o >> 13) & 4u) | ((o >> 28) & 8u)) << (4 * x);
     }
     return b;
-}
-
-// Keep bits of query i for the 128 keys [j0, j0 + 128) (j0 a multiple of
-// 128): keys 2P (bit P % 16) and 2P + 1 (bit 16 + P % 16) of keep[P / 16],
-// for the key pairs P = 0..63 of the block.
-__device__ __forceinline__ void keep_bits_row128(const DropoutParams& d, uint32_t j0, uint32_t i,
-                                                 uint32_t bh, uint32_t (&keep)[4]) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const uint32_t lo = keep_bits16(philox4x32(d, (j0 >> 4) + 2 * c, i, bh, d.offset),
-                                        d.lanes_ref);
-        const uint32_t hi = keep_bits16(philox4x32(d, (j0 >> 4) + 2 * c + 1, i, bh, d.offset),
-                                        d.lanes_ref);
-        // a call covers 8 pairs: bits 0..7 (low keys) and 16..23 (high keys)
-        keep[c] = (lo & 0x00FF00FFu) | ((hi & 0x00FF00FFu) << 8);
-    }
 }
 
 // Keep bits of one key (this lane's) against 64 consecutive queries q0 .. q0+63,
@@ -111,12 +96,8 @@ __device__ __forceinline__ unsigned long long keep_bits_key_row(const DropoutPar
     unsigned long long D = 0ull;
 #pragma unroll
     for (uint32_t m = 0; m < 4; ++m) {
-        const uint32_t b = keep_bits16(philox4x32(d, key >> 4, q0 + 16 * m + w, bh, d.offset),
-                                       d.lanes_ref);
-        // b: pair x = k / 2 at bit x (even key) and bit 16 + x (odd key)
-        uint32_t byk = 0;  // bit k = key k
-#pragma unroll
-        for (int x = 0; x < 8; ++x) byk |= ((b >> x) & 1u) << (2 * x) | ((b >> (16 + x)) & 1u) << (2 * x + 1);
+        const uint32_t byk = keep_bits16(philox4x32(d, key >> 4, q0 + 16 * m + w, bh, d.offset),
+                                         d.lanes_ref);  // bit k = key k
         D |= static_cast<unsigned long long>(byk) << (16 * m);
     }
     constexpr unsigned long long EVERY16 = 0x0001000100010001ull;
