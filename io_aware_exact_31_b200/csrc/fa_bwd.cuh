@@ -13,6 +13,10 @@
 //   1. bwd_pre:  D_i (fp32), LSE_i * log2(e), zero the fp32 dQ accumulator
 //   2. bwd_main: one CTA per (key block of 128, head); loops over query blocks
 //   3. bwd_dq:   dQ = bf16(scale * dQacc)
+// 2 and 3 are programmatic dependent launches: bwd_main's CTAs start (TMEM,
+// barriers, K/V/Q/dO loads) while bwd_pre drains and wait (griddepcontrol)
+// only before reading D, LSE2 or the accumulator; bwd_dq's CTAs wait for the
+// whole of bwd_main.  What follows the three still sees them in stream order.
 //
 // bwd_main, per query block i (the key block j is fixed per CTA):
 //   MMA1  S^T  = K_j Q_i^T            TMEM [0,128)      (lane = key)
@@ -121,6 +125,7 @@ fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __re
                   long long rows_pad, const int* __restrict__ seqlens, int H,
                   int* __restrict__ dq_count, long long n_count) {
     constexpr int TPR = D / 8;  // threads per row, 8 bf16 (16 B) each
+    grid_dep_launch();  // the main kernel may start its prologue
     const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     for (long long c = tid; c < n_count; c += static_cast<long long>(gridDim.x) * blockDim.x)
         dq_count[c] = 0;
@@ -164,6 +169,7 @@ template <int D>
 __global__ void __launch_bounds__(256)
 fa_bwd_dq_kernel(const float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dQ, int N, int Npad,
                  float scale, long long n_vec) {
+    grid_dep_wait();  // dQacc is complete only when the main kernel has finished
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_vec;
          e += stride) {
@@ -271,6 +277,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    grid_dep_launch();  // the finalize kernel waits for this grid's completion
 
     if (warp == 9) {
         // ------------------------------------------------------------ TMA producer
@@ -300,6 +307,9 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
                     tma_load_3d(smem + C::OFF_DO + s * C::TILE + c * 16384, &mapdO,
                                 &bars->q_full[s], c * 64, q0, bh);
                 }
+                // D and LSE2 come from the preprocess kernel (launched before
+                // this one, which may have started before it finished).
+                if (it == 0) grid_dep_wait();
                 const size_t voff = static_cast<size_t>(bh) * p.Npad + q0;
                 bulk_load(smem + C::OFF_VEC + s * 1024, p.LSE2 + voff, 512, &bars->q_full[s]);
                 bulk_load(smem + C::OFF_VEC + s * 1024 + 512, p.Dvec + voff, 512, &bars->q_full[s]);
@@ -408,6 +418,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         regs_decrease<BWD_REGS_CONTROL>();
         if (lane == 0) {
             tma_prefetch_desc(&mapdQacc);
+            grid_dep_wait();  // dQacc and the counters are zeroed by the preprocess kernel
             // Deterministic mode: the additions into one dQ block are made in
             // ascending key-block order.  Before adding, wait until the block's
             // counter equals this CTA's key block (every earlier key block of
@@ -718,17 +729,35 @@ bool bwd_launch_t(const void* Q, const void* K, const void* V, const void* O, co
         p.drop = drop;
         const long long n_ctas = static_cast<long long>(Npad / 128) * B * Hkv;
         if (n_ctas > 0x7fffffffLL) return false;
-        dim3 grid(static_cast<unsigned>(n_ctas));
-        fa_bwd_main_kernel<D, DROP><<<grid, BWD_THREADS, BwdCfg<D>::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mdo, mdq, p);
-        if (cudaGetLastError() != cudaSuccess) return false;
+        cudaLaunchAttribute pdl[1];
+        pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pdl[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
+        cfg.blockDim = dim3(BWD_THREADS);
+        cfg.dynamicSmemBytes = BwdCfg<D>::SMEM_BYTES;
+        cfg.stream = stream;
+        cfg.attrs = pdl;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, fa_bwd_main_kernel<D, DROP>, mq, mk, mv, mdo, mdq, p) !=
+            cudaSuccess)
+            return false;
     }
     {
         const long long n_vec = static_cast<long long>(B) * H * N * (D / 8);
         const int blocks = static_cast<int>(std::min<long long>((n_vec + 255) / 256, 148LL * 16));
-        fa_bwd_dq_kernel<D><<<blocks, 256, 0, stream>>>(dQacc, static_cast<__nv_bfloat16*>(dQ), N,
-                                                        Npad, scale, n_vec);
-        if (cudaGetLastError() != cudaSuccess) return false;
+        cudaLaunchAttribute pdl[1];
+        pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pdl[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(blocks);
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cfg.attrs = pdl;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, fa_bwd_dq_kernel<D>, static_cast<const float*>(dQacc),
+                               static_cast<__nv_bfloat16*>(dQ), N, Npad, scale, n_vec) != cudaSuccess)
+            return false;
     }
     return true;
 }
