@@ -463,7 +463,7 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         const uint32_t sDQ = smem_u32(smem + C::OFF_DQ);
         float pv[64];  // P^T (then dS^T) for this thread's 64 queries
         uint32_t keep_lo = ~0u, keep_hi = ~0u;  // dropout keep bits of those queries
-        auto kept = [&](int c) { return (((c < 32) ? keep_lo : keep_hi) >> (c & 31)) & 1u; };
+        auto kept = [&](int c) { return (((c < 32) ? keep_lo : keep_hi) >> keep_bit_index(c & 31)) & 1u; };
         bool ok = true;
 
         // ---- P(it): P^T = exp2(S^T * scale*log2e - LSE2[q])
@@ -474,11 +474,11 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
             const int qh = q0 + 64 * half;  // first query of this warp's columns
             if constexpr (DROP) {
                 // Made before S^T is ready: they depend only on the indices.
-                const unsigned long long M = keep_bits_key_row(
-                    p.drop, static_cast<uint32_t>(key), static_cast<uint32_t>(qh),
-                    static_cast<uint32_t>(q_head(it)), lane);
-                keep_lo = static_cast<uint32_t>(M);
-                keep_hi = static_cast<uint32_t>(M >> 32);
+                const uint2 M = keep_bits_key_row(p.drop, static_cast<uint32_t>(key),
+                                                  static_cast<uint32_t>(qh),
+                                                  static_cast<uint32_t>(q_head(it)), lane);
+                keep_lo = M.x;
+                keep_hi = M.y;
             }
             if (!mbar_wait(&bars->q_full[s], ph, g, 29)) return false;
             if (!mbar_wait_warp(&bars->s_full, it & 1, g, 30)) return false;

@@ -519,8 +519,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                             // where its integer work overlaps the exponentials;
                             // the pair's bytes sit in the two 16-bit lanes of
                             // word (i % 8) / 2 (bytes 0/2 for even i, 1/3 for odd
-                            // i), and keep_lanes turns each lane's decision into
-                            // bit 15 / bit 31, spread here to a 16-bit mask.
+                            // i); keep_mask16 turns the two decisions into the
+                            // 16-bit masks of the pair.
                             if (i % 8 == 0)
                                 dw = philox4x32(p.drop,
                                                 static_cast<uint32_t>((j * FWD_BN) / 16 + 4 * h + i / 8),
@@ -530,9 +530,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                                                 : ((i % 8) / 2 == 1) ? dw.y
                                                 : ((i % 8) / 2 == 2) ? dw.z
                                                                      : dw.w;
-                            const uint32_t lanes =
-                                (i % 2 == 0) ? (wd & 0x00FF00FFu) : ((wd >> 8) & 0x00FF00FFu);
-                            pk[i] &= (keep_lanes(lanes, p.drop.lanes_ref) >> 15) * 0xFFFFu;
+                            pk[i] &= keep_mask16(byte_lanes(wd, i % 2 == 0), p.drop.lanes_ref);
                         }
                     }
                 }
