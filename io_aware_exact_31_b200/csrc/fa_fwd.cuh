@@ -292,11 +292,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
 
             // S_t = Q_t K_j^T : K-major A and B, steps of 32 bytes along d.
             auto issue_S = [&](int t, int s) {
+                const uint64_t a0 = sdesc_sw128(sQ + t * C::TILE_BYTES, 16, 1024);
+                const uint64_t b0 = sdesc_sw128(sK + s * C::TILE_BYTES, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / C::KSTEP; ++kk) {
-                    const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
-                    const uint64_t a = sdesc_sw128(sQ + t * C::TILE_BYTES + koff, 16, 1024);
-                    const uint64_t b = sdesc_sw128(sK + s * C::TILE_BYTES + koff, 16, 1024);
+                    const uint32_t ko = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
+                    const uint64_t a = desc_off(a0, ko);
+                    const uint64_t b = desc_off(b0, ko);
                     if constexpr (F8) mma_ss_f8_w(tS[t], a, b, idS, kk > 0);
                     else mma_ss_w(tS[t], a, b, idS, kk > 0);
                 }
@@ -306,11 +308,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             // The two halves are issued as soon as the softmax warps release
             // each half of P.
             auto issue_PV_half = [&](int t, int s, int h, bool acc) {
+                const uint64_t b0 = sdesc_sw128(sV + s * C::TILE_BYTES, 16384, 1024);
 #pragma unroll
                 for (int i = 0; i < C::PV_PER_HALF; ++i) {
                     const int kk = h * C::PV_PER_HALF + i;
-                    const uint64_t b = sdesc_sw128(sV + s * C::TILE_BYTES + kk * C::KSTEP * 128,
-                                                   16384, 1024);
+                    const uint64_t b = desc_off(b0, (kk * C::KSTEP * 128) >> 4);
                     if constexpr (F8) mma_ts_f8_w(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
                     else mma_ts_w(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
                 }

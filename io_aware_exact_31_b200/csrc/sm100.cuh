@@ -357,6 +357,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
            | (2ull << 61);                                                       // SWIZZLE_128B
 }
 
+// Descriptor d advanced by k 16-byte units: added to the start-address field
+// (bits 0-13) in the low word only, which cannot carry while the shared
+// address stays below 2^18.
+__device__ __forceinline__ uint64_t desc_off(uint64_t d, uint32_t k) {
+    const uint32_t lo = static_cast<uint32_t>(d) + k;
+    return (d & 0xFFFFFFFF00000000ull) | lo;
+}
+
 // Instruction descriptor, kind::f8f6f4 with E4M3 A/B and fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_e4m3(uint32_t M, uint32_t N, bool b_mn) {
     return (1u << 4)                        // D format: f32

@@ -131,7 +131,7 @@ def test_extended_entry_points_reject_bad_arguments_without_a_device(lib):
     assert lib.fa_forward_gqa(*a, 1, 4, 0, 8, 64, 0.125, 0, None) == INV
     # padded batches: seqlens must be 4-byte aligned
     assert lib.fa_forward_varlen(*a, 18, 1, 2, 2, 8, 64, 0.125, 0, None) == INV
-    # dropout: p in [0, 1 - 2^-16]
+    # dropout: p in [0, 1 - 2^-9]
     for pd in (1.0, -0.1, float("nan"), 1.0 - 2.0 ** -17):
         assert lib.fa_forward_dropout(*a, None, 1, 2, 2, 8, 64, 0.125, 0, pd, 1, 0, None) == INV
     assert lib.fa_forward_dropout(None, *a[1:], None, 1, 2, 2, 8, 64, 0.125, 0, 0.1, 1, 0,
