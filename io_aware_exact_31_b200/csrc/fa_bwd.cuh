@@ -338,29 +338,18 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
                 // reuse of S^T / P^T: S^T(it+1) follows dV(it), which followed
                 // P^T(it) being written, i.e. S^T(it) being read.
                 auto mma_S = [&](int it) {  // S^T = K Q^T
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
-                        mma_ss_w(tmem + C::T_ST, sdesc_sw128(sK + ko, 16, 1024),
-                               sdesc_sw128(sQ(it) + ko, 16, 1024), id_s, kk > 0);
-                    }
+                    mma_ss_blk<D / 16, FA_STEP_KMAJOR, FA_STEP_KMAJOR>(
+                        tmem + C::T_ST, sdesc_sw128(sK, 16, 1024), sdesc_sw128(sQ(it), 16, 1024), id_s, 0u);
                     tc_commit_w(&bars->s_full);
                 };
                 auto mma_dP = [&](int it) {  // dP^T = V dO^T
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t ko = (kk / 4) * 16384 + (kk % 4) * 32;
-                        mma_ss_w(tmem + C::T_DPT, sdesc_sw128(sV + ko, 16, 1024),
-                               sdesc_sw128(sdO(it) + ko, 16, 1024), id_s, kk > 0);
-                    }
+                    mma_ss_blk<D / 16, FA_STEP_KMAJOR, FA_STEP_KMAJOR>(
+                        tmem + C::T_DPT, sdesc_sw128(sV, 16, 1024), sdesc_sw128(sdO(it), 16, 1024), id_s, 0u);
                     tc_commit_w(&bars->dp_full);
                 };
                 auto mma_dV = [&](int it) {  // dV += P^T dO   (P^T from TMEM)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts_w(tmem + C::T_DV, tmem + C::T_PT + kk * 8,
-                               sdesc_sw128(sdO(it) + kk * 2048, 16384, 1024), id_kn,
-                               (it > 0 || kk > 0));
+                    mma_ts_blk<8, 8, 128>(tmem + C::T_DV, tmem + C::T_PT,
+                                          sdesc_sw128(sdO(it), 16384, 1024), id_kn, it > 0 ? 1u : 0u);
                     tc_commit_w(&bars->q_empty[it % C::QS]);  // this issuer is done with the stage
                 };
                 bool ok = mbar_wait_warp(&bars->kv_full, 0, g, 22) && q_wait(0, 23);
@@ -398,14 +387,13 @@ fa_bwd_main_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
                         break;
                     // ...or dP^T(it), which ds_full shows read (d = 128).
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // dK += dS^T Q
-                        mma_ss_w(tmem + C::T_DK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
-                               sdesc_sw128(sQ(it) + kk * 2048, 16384, 1024), id_kn, (it > 0 || kk > 0));
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // dQ = dS K
-                        mma_ss_w(tmem + C::T_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
-                               sdesc_sw128(sK + kk * 2048, 16384, 1024), id_q, kk > 0);
+                    // dK += dS^T Q
+                    mma_ss_blk<8, FA_STEP_KMAJOR, 128>(tmem + C::T_DK, sdesc_sw128(sDS, 16, 1024),
+                                                       sdesc_sw128(sQ(it), 16384, 1024), id_kn,
+                                                       it > 0 ? 1u : 0u);
+                    // dQ = dS K
+                    mma_ss_blk<8, 128, 128>(tmem + C::T_DQ, sdesc_sw128(sDS, 16384, 1024),
+                                            sdesc_sw128(sK, 16384, 1024), id_q, 0u);
                     tc_commit_w(&bars->dq_full);
                     tc_commit_w(&bars->ds_empty);
                     tc_commit_w(&bars->q_empty[it % C::QS]);

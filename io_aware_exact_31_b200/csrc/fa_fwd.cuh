@@ -38,9 +38,9 @@
 // (barrier s_free) -- so it is computed while the exponentials of block j
 // run, and the per-tile chain S -> softmax -> P.V -> S is broken.  Three
 // threads issue the MMAs: warp 8 all S_t, warps 10 and 11 the P.V of tile 0
-// and tile 1 (one thread issues an MMA only every ~110-130 clocks whatever
-// its size, and at d = 64 most of the MMAs are small).  The softmax waits for
-// P.V_t(j-1) (barrier pv_done) before it rescales O_t or overwrites P_t.
+// and tile 1, so that each issuing thread waits only on the barriers of its
+// own instructions.  The softmax waits for P.V_t(j-1)
+// (barrier pv_done) before it rescales O_t or overwrites P_t.
 #pragma once
 
 #include "philox.cuh"
@@ -212,12 +212,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                             // descriptor of this V stage; k-steps advance its
                             // address field (16-byte units, no carry: < 256 KB)
                             const uint64_t b0 = sdesc_sw128(sV + sv * C::TILE_BYTES, 16384, 1024);
-#pragma unroll
-                            for (int i = 0; i < C::PV_PER_HALF; ++i) {
-                                const int kk = h * C::PV_PER_HALF + i;
-                                mma_ts_w(tO, tP + kk * 8, b0 + (kk * C::KSTEP * 128 >> 4), idO,
-                                         (j > 0 || kk > 0) ? 1u : 0u);
-                            }
+                            const int kk0 = h * C::PV_PER_HALF;
+                            mma_ts_blk<C::PV_PER_HALF, 8, C::KSTEP * 8>(
+                                tO, tP + kk0 * 8, desc_off(b0, kk0 * C::KSTEP * 8), idO,
+                                (j > 0 || h > 0) ? 1u : 0u);
                         }
                         if (!ok) break;
                         tc_commit_w(&bars->pv_done[t]);
@@ -294,14 +292,10 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             auto issue_S = [&](int t, int s) {
                 const uint64_t a0 = sdesc_sw128(sQ + t * C::TILE_BYTES, 16, 1024);
                 const uint64_t b0 = sdesc_sw128(sK + s * C::TILE_BYTES, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < D / C::KSTEP; ++kk) {
-                    const uint32_t ko = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4;
-                    const uint64_t a = desc_off(a0, ko);
-                    const uint64_t b = desc_off(b0, ko);
-                    if constexpr (F8) mma_ss_f8_w(tS[t], a, b, idS, kk > 0);
-                    else mma_ss_w(tS[t], a, b, idS, kk > 0);
-                }
+                if constexpr (F8)
+                    mma_ss_f8_blk<D / C::KSTEP, FA_STEP_KMAJOR, FA_STEP_KMAJOR>(tS[t], a0, b0, idS, 0u);
+                else
+                    mma_ss_blk<D / C::KSTEP, FA_STEP_KMAJOR, FA_STEP_KMAJOR>(tS[t], a0, b0, idS, 0u);
             };
             // O_t (+)= P_t V_j for keys [64h, 64h + 64): P from TMEM (8 columns
             // per instruction), V MN-major (KSTEP key rows of 128 B per step).
@@ -309,13 +303,13 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             // each half of P.
             auto issue_PV_half = [&](int t, int s, int h, bool acc) {
                 const uint64_t b0 = sdesc_sw128(sV + s * C::TILE_BYTES, 16384, 1024);
-#pragma unroll
-                for (int i = 0; i < C::PV_PER_HALF; ++i) {
-                    const int kk = h * C::PV_PER_HALF + i;
-                    const uint64_t b = desc_off(b0, (kk * C::KSTEP * 128) >> 4);
-                    if constexpr (F8) mma_ts_f8_w(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
-                    else mma_ts_w(tO[t], tS[t] + kk * 8, b, idO, (acc || kk > 0) ? 1u : 0u);
-                }
+                const int kk0 = h * C::PV_PER_HALF;
+                const uint64_t b = desc_off(b0, kk0 * C::KSTEP * 8);
+                const uint32_t en = (acc || h > 0) ? 1u : 0u;
+                if constexpr (F8)
+                    mma_ts_f8_blk<C::PV_PER_HALF, 8, C::KSTEP * 8>(tO[t], tS[t] + kk0 * 8, b, idO, en);
+                else
+                    mma_ts_blk<C::PV_PER_HALF, 8, C::KSTEP * 8>(tO[t], tS[t] + kk0 * 8, b, idO, en);
             };
 
             bool ok = mbar_wait_warp(&bars->q_full, 0, g, 3);

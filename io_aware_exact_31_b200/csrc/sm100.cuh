@@ -325,14 +325,6 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulator.
 // a_mn / b_mn select MN-major (transposed) operands in shared memory.
 __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N, bool a_mn, bool b_mn) {
@@ -373,89 +365,87 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(uint32_t M, uint32_t N, bool b
            | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-            d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+// MMA issue.  The whole warp, converged, executes the call; elect.sync inside
+// the instruction block picks one lane (the same lane every time in a fully
+// converged warp, so tc_commit_w tracks the MMAs that lane issued).  NSTEP
+// K-steps of one accumulation go out from a single inline-PTX block with one
+// elect.sync.  Step k > 0 reads the operands at the base descriptors advanced by
+// a compile-time number of 16-byte units (added to the start-address field,
+// which cannot carry below 256 KB of shared memory); the first step accumulates
+// when `acc` is non-zero, the others always do.
+//
+// Issued this way one warp keeps the tensor core at its full rate: M = 128,
+// N = 128, K = 16 bf16 MMAs complete every ~64 clocks whether A comes from
+// shared memory or TMEM, also in the forward's sequence of two P.V halves and
+// an S (with other warps streaming tcgen05.ld / st or exponentials meanwhile),
+// and N = 64 ones every ~42-48.  One elect.sync block per MMA costs ~94 (SS) /
+// ~104 (TS) clocks per instruction whatever N is up to 128, and a lane-0 branch
+// of a diverged warp ~140 (microbenchmarks on B200, 148 SMs, one issuing warp
+// per SM).
+//
+// Offset patterns (16-byte units at step k):
+//   FA_STEP_KMAJOR (0): K-major 128-byte-swizzled tile, 32-byte K-steps inside
+//                       128-byte rows, 64-element (bf16) row chunks 16 KB apart;
+//   P > 0:              P units per step (MN-major tiles: K rows of 128 bytes).
+#define FA_STEP_KMAJOR 0
+template <int P>
+__host__ __device__ constexpr uint32_t blk_off(int k) {
+    return P == FA_STEP_KMAJOR ? static_cast<uint32_t>((k / 4) * 1024 + (k % 4) * 2)
+                               : static_cast<uint32_t>(k * P);
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T  (A: lane = row, bf16 pairs packed per column)
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-            d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
-}
-
-// 8-bit (E4M3) operand versions: k = 32 elements (32 bytes) per instruction.
-__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-            d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
-}
-
-// A from TMEM: four E4M3 values per 32-bit column (element 4c + b in byte b).
-__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(
-            d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
-}
-
-// Warp-collective forms of the MMA and commit above.  The whole warp, converged,
-// executes the call; elect.sync inside the instruction block picks one lane
-// (the same lane every time in a fully converged warp, so the commit tracks
-// the MMAs that lane issued).  Issued this way a single warp sends
-// back-to-back M = 128, N = 128, K = 16 MMAs every ~94 (shared-memory A) /
-// ~105 (TMEM A) clocks and N = 256 ones at the tensor core's full rate,
-// against ~140 clocks per instruction from a lane-0 branch of a diverged warp
-// (microbenchmark on B200, 148 SMs, one issuing warp per SM).
-#define FA_ELECT_MMA(kind, aop)                                                        \
-    "{\n\t.reg .pred p, e;\n\t"                                                          \
+#define FA_BLK_HEAD                                                                    \
+    "{\n\t.reg .pred p, q, e;\n\t.reg .b64 a, b;\n\t.reg .b32 t;\n\t"                    \
     "elect.sync _|e, 0xffffffff;\n\t"                                                    \
     "setp.ne.b32 p, %4, 0;\n\t"                                                          \
-    "@e tcgen05.mma.cta_group::1.kind::" kind " [%0], " aop ", %2, %3, p;\n\t}"
+    "setp.eq.b32 q, %4, %4;\n\t"
+#define FA_SS0(K) "@e tcgen05.mma.cta_group::1.kind::" K " [%0], %1, %2, %3, p;\n\t"
+#define FA_SSN(K, OA, OB)                                                              \
+    "add.s64 a, %1, " OA ";\n\tadd.s64 b, %2, " OB ";\n\t"                             \
+    "@e tcgen05.mma.cta_group::1.kind::" K " [%0], a, b, %3, q;\n\t"
+#define FA_TS0(K) "@e tcgen05.mma.cta_group::1.kind::" K " [%0], [%1], %2, %3, p;\n\t"
+#define FA_TSN(K, OA, OB)                                                              \
+    "add.s32 t, %1, " OA ";\n\tadd.s64 b, %2, " OB ";\n\t"                             \
+    "@e tcgen05.mma.cta_group::1.kind::" K " [%0], [t], b, %3, q;\n\t"
 
-__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
-    asm volatile(FA_ELECT_MMA("f16", "%1")::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc),
-                 "r"(accumulate));
-}
+#define FA_IN5_SS "r"(d), "l"(a0), "l"(b0), "r"(id), "r"(acc)
+#define FA_IN5_TS "r"(d), "r"(a0), "l"(b0), "r"(id), "r"(acc)
+#define FA_OFF2(F, G) "n"(F(1)), "n"(G(1))
+#define FA_OFF4(F, G) "n"(F(1)), "n"(F(2)), "n"(F(3)), "n"(G(1)), "n"(G(2)), "n"(G(3))
+#define FA_OFF8(F, G)                                                                  \
+    "n"(F(1)), "n"(F(2)), "n"(F(3)), "n"(F(4)), "n"(F(5)), "n"(F(6)), "n"(F(7)),       \
+        "n"(G(1)), "n"(G(2)), "n"(G(3)), "n"(G(4)), "n"(G(5)), "n"(G(6)), "n"(G(7))
 
-__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
-    asm volatile(FA_ELECT_MMA("f16", "[%1]")::"r"(d_tmem), "r"(a_tmem), "l"(b_desc),
-                 "r"(idesc), "r"(accumulate));
-}
+#define FA_DEFINE_BLK(NAME, KIND, ATYPE, S0, SN, IN5)                                          \
+    template <int NSTEP, int PA, int PB>                                                  \
+    __device__ __forceinline__ void NAME(uint32_t d, ATYPE a0, uint64_t b0, uint32_t id,  \
+                                         uint32_t acc) {                                  \
+        static_assert(NSTEP == 2 || NSTEP == 4 || NSTEP == 8, "NSTEP must be 2, 4 or 8"); \
+        if constexpr (NSTEP == 2) {                                                       \
+            asm volatile(FA_BLK_HEAD S0(KIND) SN(KIND, "%5", "%6") "}" ::IN5,          \
+                         FA_OFF2(blk_off<PA>, blk_off<PB>));                              \
+        } else if constexpr (NSTEP == 4) {                                                \
+            asm volatile(FA_BLK_HEAD S0(KIND) SN(KIND, "%5", "%8") SN(KIND, "%6", "%9")  \
+                             SN(KIND, "%7", "%10") "}" ::IN5,                          \
+                         FA_OFF4(blk_off<PA>, blk_off<PB>));                              \
+        } else {                                                                          \
+            asm volatile(FA_BLK_HEAD S0(KIND) SN(KIND, "%5", "%12") SN(KIND, "%6", "%13") \
+                             SN(KIND, "%7", "%14") SN(KIND, "%8", "%15")                  \
+                                 SN(KIND, "%9", "%16") SN(KIND, "%10", "%17")             \
+                                     SN(KIND, "%11", "%18") "}" ::IN5,                 \
+                         FA_OFF8(blk_off<PA>, blk_off<PB>));                              \
+        }                                                                                 \
+    }
 
-__device__ __forceinline__ void mma_ss_f8_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(FA_ELECT_MMA("f8f6f4", "%1")::"r"(d_tmem), "l"(a_desc), "l"(b_desc),
-                 "r"(idesc), "r"(accumulate));
-}
+// D (+)= A[smem] B[smem]^T, NSTEP K-steps; PA / PB: offset patterns of A and B.
+FA_DEFINE_BLK(mma_ss_blk, "f16", uint64_t, FA_SS0, FA_SSN, FA_IN5_SS)
+FA_DEFINE_BLK(mma_ss_f8_blk, "f8f6f4", uint64_t, FA_SS0, FA_SSN, FA_IN5_SS)
+// D (+)= A[tmem] B[smem]^T, NSTEP K-steps; A advances by PA columns per step.
+FA_DEFINE_BLK(mma_ts_blk, "f16", uint32_t, FA_TS0, FA_TSN, FA_IN5_TS)
+FA_DEFINE_BLK(mma_ts_f8_blk, "f8f6f4", uint32_t, FA_TS0, FA_TSN, FA_IN5_TS)
 
-__device__ __forceinline__ void mma_ts_f8_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(FA_ELECT_MMA("f8f6f4", "[%1]")::"r"(d_tmem), "r"(a_tmem), "l"(b_desc),
-                 "r"(idesc), "r"(accumulate));
-}
-
-// Warp-collective tc_commit (the elected lane is the one that issued the MMAs).
+// Arrive once on `bar` when every tcgen05 op issued so far by the elected lane
+// (the one that issued the MMAs) is done.  Warp-collective.
 __device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
