@@ -117,7 +117,7 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
                          float scale, int causal, cudaStream_t stream, double scale_qk = 1.0,
                          float scale_v = 1.f, const DropoutParams* drop = nullptr) {
     using C = FwdCfg<D, F8>;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     const uint64_t depth = static_cast<uint64_t>(B) * H;
     const uint64_t depth_kv = static_cast<uint64_t>(B) * Hkv;
     const bool maps_ok =
@@ -127,7 +127,8 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
            : (make_map_bf16_3d(&mq, Q, depth, N, D, FWD_BM) &&
               make_map_bf16_3d(&mk, K, depth_kv, N, D, FWD_BN) &&
               make_map_bf16_3d(&mv, V, depth_kv, N, D, FWD_BN));
-    if (!maps_ok) return FA_ERR_CUDA;
+    // O (bf16 in every variant) is written by TMA stores of Q-shaped tiles.
+    if (!maps_ok || !make_map_bf16_3d(&mo, O, depth, N, D, FWD_BM)) return FA_ERR_CUDA;
     const int di = F8 ? 2 : ((D == 128) ? 1 : 0) + (DROP ? 3 : 0);
     {
         std::lock_guard<std::mutex> lock(g_mu);
@@ -161,7 +162,7 @@ fa_status launch_forward(DeviceState* ds, const void* Q, const void* K, const vo
     const long long n_ctas = static_cast<long long>(p.n_pairs) * p.n_heads;
     if (n_ctas > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
     dim3 grid(static_cast<unsigned>(n_ctas));
-    fa_fwd_kernel<D, F8, DROP><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+    fa_fwd_kernel<D, F8, DROP><<<grid, FWD_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -116,7 +116,8 @@ static_assert(sizeof(FwdBars) + 8 <= 256, "barrier area");
 template <int D, bool F8 = false, bool DROP = false>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-              const __grid_constant__ CUtensorMap mapV, const FwdParams p) {
+              const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapO,
+              const FwdParams p) {
     static_assert(!(F8 && DROP), "dropout is implemented for bf16 operands only");
     using C = FwdCfg<D, F8>;
     extern __shared__ uint8_t smem_raw[];
@@ -566,32 +567,76 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 for (int c = 0; c < D; c += 8) st_global_v4(orow + c, 0u, 0u, 0u, 0u);
                 p.LSE[static_cast<size_t>(bh) * p.N + q] = 0.f;
             }
-        } else if (ok && (C::SEP ? mbar_wait_warp(&bars->pv_done[t], (nt - 1) & 1, g, 25 + t)
-                                 : mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t))) {
-            tc_fence_after();
+        } else {
+            // O_t is complete once its last P.V is (every warp waits; the tile's
+            // four warps then meet at a named barrier whatever the outcome).
+            const bool go = ok && (C::SEP ? mbar_wait_warp(&bars->pv_done[t], (nt - 1) & 1, g, 25 + t)
+                                          : mbar_wait_warp(&bars->o_full[t], 0, g, 11 + t));
+            if (go) tc_fence_after();
             const bool real = q < len;  // padding rows of a partly padded tile get zeros
             const float inv_l = real ? p.o_scale / lr : 0.f;
             const bool valid = q < p.N;
-            __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + (valid ? q : 0)) * D;
+            if constexpr (!F8) {
+                // O_t out of TMEM in one go, normalised, packed to bf16 and
+                // written in the 128-byte-swizzled layout of a Q tile into Q_t's
+                // own shared memory, which no MMA reads once O_t is complete
+                // (its last S was issued before its last P.V, by the same
+                // thread or, with P in its own columns, read by this softmax).
+                // One thread then writes the tile with TMA stores, which clip
+                // the rows past N.
+                uint8_t* stage = smem + C::OFF_Q + t * C::TILE_BYTES;
+                if (go) {
+                    uint32_t o[D];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, o + c * 32);
+                    tmem_ld_wait();
+                    reg_fence<D>(o);
+                    const uint32_t srow = smem_u32(stage) + static_cast<uint32_t>(row) * 128u;
+#pragma unroll
+                    for (int u = 0; u < D / 8; ++u) {  // 16-byte units: 8 columns each
+                        const uint32_t chunk = u / 8, uu = u % 8;
+                        st_shared_v4(srow + chunk * 16384u + ((uu ^ (static_cast<uint32_t>(row) & 7u)) << 4),
+                                     pack_bf16x2(__uint_as_float(o[8 * u + 0]) * inv_l,
+                                                 __uint_as_float(o[8 * u + 1]) * inv_l),
+                                     pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv_l,
+                                                 __uint_as_float(o[8 * u + 3]) * inv_l),
+                                     pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv_l,
+                                                 __uint_as_float(o[8 * u + 5]) * inv_l),
+                                     pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv_l,
+                                                 __uint_as_float(o[8 * u + 7]) * inv_l));
+                    }
+                    fence_proxy_async_smem();
+                }
+                const bool tile_go = named_bar_and(1 + t, 128, go);  // the tile's four warps
+                if (tile_go && warp % 4 == 0 && lane == 0) {
+#pragma unroll
+                    for (int c = 0; c < C::CHUNKS; ++c)
+                        tma_store_3d(&mapO, stage + c * 16384, c * C::BOX_ELEMS, tile_first_q, bh);
+                    bulk_commit_group();
+                    bulk_wait_read_all();  // shared memory read before the CTA exits
+                }
+            } else if (go) {
+                __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + (valid ? q : 0)) * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + c * 32, o);
-                tmem_ld_wait();
-                reg_fence<32>(o);
-                uint32_t w[16];
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_ld_wait();
+                    reg_fence<32>(o);
+                    uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
-                                       __uint_as_float(o[2 * i + 1]) * inv_l);
-                if (valid) {
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                                           __uint_as_float(o[2 * i + 1]) * inv_l);
+                    if (valid) {
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        st_global_v4(orow + c * 32 + v * 8, w[4 * v], w[4 * v + 1], w[4 * v + 2],
-                                     w[4 * v + 3]);
+                        for (int v = 0; v < 4; ++v)
+                            st_global_v4(orow + c * 32 + v * 8, w[4 * v], w[4 * v + 1], w[4 * v + 2],
+                                         w[4 * v + 3]);
+                    }
                 }
             }
-            if (valid) {
+            if (go && valid) {
                 // LSE in natural-log units: (m + log2 l) * ln 2.
                 p.LSE[static_cast<size_t>(bh) * p.N + q] =
                     real ? (m_used + __log2f(l)) * 0.69314718055994531f : 0.f;
