@@ -28,10 +28,9 @@
 // accumulator with TMA tensor reduce-adds (one per 32-column box).
 // Warps: 0-7 compute (warp w: TMEM lane quarter w%4, column half w/4),
 // 8 MMA issuer of S^T, dP^T and dV (TMEM owner), 9 TMA producer, 10 dQ
-// reducer, 11 MMA issuer of dK and dQ.  One thread issues a tcgen05.mma only
-// about every 110 clocks whatever its size, and at d = 64 three of the five
-// products have N = 64, so a single issuer would leave the tensor core idle
-// most of the time; two issuers share the 5 products 16 : 16 instructions.
+// reducer, 11 MMA issuer of dK and dQ.  The two issuers share the five
+// products 16 : 16 instructions, so that S^T(i+1) is not held behind the
+// barrier waits of dK(i) and dQ(i).
 #pragma once
 
 #include <algorithm>
