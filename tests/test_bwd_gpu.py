@@ -36,6 +36,14 @@ def test_b4_h16_n2048_d64_causal_sampled_heads():
     check_backward(w.B, w.H, w.N, w.d, w.causal, heads=ends + pick)
 
 
+def test_b4_h16_n2048_d128_causal_sampled_heads():
+    """The backward at head dimension 128 on the same shape (the benchmark's
+    --bwd-d 128 run): the first and last head of every batch."""
+    w = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
+    heads = [(b, h) for b in range(w.B) for h in (0, w.H - 1)]
+    check_backward(w.B, w.H, w.N, 128, True, seed=0, heads=heads)
+
+
 def test_autograd_wrapper_matches_raw():
     x = inputs(1, 2, 200, 64, seed=13, with_dO=True)
     q, k, v, do = (x[n].cuda() for n in ("Q", "K", "V", "dO"))
