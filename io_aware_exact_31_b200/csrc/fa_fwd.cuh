@@ -429,8 +429,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     if (key0 + i >= lim) s[i] = -INFINITY;
             }
             // Row max: eight independent three-input chains (short dependency depth).
-            float mx;
-            {
+            auto row_max = [&]() {
                 float a[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) a[k] = fmaxf(s[2 * k], s[2 * k + 1]);
@@ -438,19 +437,30 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 for (int i = 16; i < 128; i += 16)
 #pragma unroll
                     for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[i + 2 * k], s[i + 2 * k + 1]);
-                mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7]));
-            }
-            const float m_blk = mx * sl2;
+                return fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7]));
+            };
+            // With P in its own columns (and no dropout, whose kernel would
+            // spill with both paths) the blocks after the first skip the row
+            // max: their weights are taken against the running reference as it
+            // stands, and only a block whose weights reach 2^64 against it
+            // (checked on the row sum below) is redone against its own max.
+            // O and l stay exact either way (one reference for both); 2^64
+            // keeps every fp32 accumulation far from overflow.
+            constexpr bool kLazyMax = C::SEP && !DROP;
+            const bool lazy_max = kLazyMax && j > 0;
             float alpha = 1.f;
-            if (j == 0) {
-                m_used = m_blk;
-            } else if (m_blk > m_used + FWD_RESCALE_TAU) {
-                alpha = ex2_approx(m_used - m_blk);
-                m_used = m_blk;
+            if (!lazy_max) {
+                const float m_blk = row_max() * sl2;
+                if (j == 0) {
+                    m_used = m_blk;
+                } else if (m_blk > m_used + FWD_RESCALE_TAU) {
+                    alpha = ex2_approx(m_used - m_blk);
+                    m_used = m_blk;
+                }
             }
             // A row whose keys are all masked so far keeps m = -inf; use 0 so
             // exp2(-inf - 0) = 0 instead of NaN.
-            const float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+            float m_sub = (m_used == -INFINITY) ? 0.f : m_used;
             // Rescale O_t in place when this row's max moved (rare after the
             // first blocks).  PV_t(j-1) must be complete: with P over S it was
             // issued before S_t(j), whose commit we waited for; with P in its
@@ -481,13 +491,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
             // P goes to TMEM as bf16 pairs (key 2c in the low half of column c),
             // or for E4M3 operands four per column (key 4c + b in byte b).
             // Packed f32x2 arithmetic, four independent accumulators per sum.
-            const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(-m_sub, -m_sub);
+            const float2 sl2v = make_float2(sl2, sl2);
             float2 ae[4], ar[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) ae[k] = ar[k] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
+            // The weights of keys [64h, 64h + 64) into pk, both row sums into ae / ar.
+            auto exp_half = [&](int h, float msub, uint32_t (&pk)[32]) {
+                const float2 negm = make_float2(-msub, -msub);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float2 x =
@@ -531,24 +539,77 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                         }
                     }
                 }
-                if constexpr (C::SEP) {
-                    if (h == 0) {
-                        // P_t and O_t are free once P.V_t(j-1) has completed.
-                        if (j > 0) {
-                            if (!(ok = mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, g, 23 + t)))
-                                break;
-                            tc_fence_after();
-                        }
-                        rescale_O();
-                    }
-                }
+            };
+            auto store_P = [&](int h, const uint32_t (&pk)[32]) {
                 if constexpr (F8) tmem_st16(tP + h * C::P_COLS_HALF, pk);
                 else tmem_st32(tP + h * C::P_COLS_HALF, pk);
-                // Release this half of P: the tensor core starts on keys
-                // [64h, 64h + 64) while the other half is still being computed.
+            };
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ae[k] = ar[k] = make_float2(0.f, 0.f);
+            if (kLazyMax && lazy_max) {
+                // Against the running reference; P_t and O_t are free once
+                // P.V_t(j-1) has completed.  Both halves are released together
+                // after the overflow check.
+                m_used = m_sub;
+                {
+                    uint32_t pk[32];
+                    exp_half(0, m_sub, pk);
+                    if (!(ok = mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, g, 23 + t))) break;
+                    tc_fence_after();
+                    store_P(0, pk);
+                    exp_half(1, m_sub, pk);
+                    store_P(1, pk);
+                }
+                const float2 e0 = __fadd2_rn(__fadd2_rn(ae[0], ae[1]), __fadd2_rn(ae[2], ae[3]));
+                if (__any_sync(0xffffffffu, !(e0.x + e0.y <= 0x1p64f))) {
+                    // Rare: this block outgrows the reference.  Move the
+                    // reference to the block's max (for every row of the warp,
+                    // as an ordinary rescale) and redo the block.
+                    const float m_blk = row_max() * sl2;
+                    if (m_blk > m_used) {
+                        alpha = ex2_approx(m_used - m_blk);
+                        m_used = m_blk;
+                    }
+                    m_sub = (m_used == -INFINITY) ? 0.f : m_used;
+                    rescale_O();
+                    l *= alpha;
+                    lr *= alpha;
+                    tmem_st_wait();  // the stores above land before their replacements
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) ae[k] = ar[k] = make_float2(0.f, 0.f);
+                    uint32_t pk[32];
+                    exp_half(0, m_sub, pk);
+                    store_P(0, pk);
+                    exp_half(1, m_sub, pk);
+                    store_P(1, pk);
+                }
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&bars->p_full[t][h]);
+                mbar_arrive(&bars->p_full[t][0]);
+                mbar_arrive(&bars->p_full[t][1]);
+            } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[32];
+                    exp_half(h, m_sub, pk);
+                    if constexpr (C::SEP) {
+                        if (h == 0) {
+                            // P_t and O_t are free once P.V_t(j-1) has completed.
+                            if (j > 0) {
+                                if (!(ok = mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, g, 23 + t)))
+                                    break;
+                                tc_fence_after();
+                            }
+                            rescale_O();
+                        }
+                    }
+                    store_P(h, pk);
+                    // Release this half of P: the tensor core starts on keys
+                    // [64h, 64h + 64) while the other half is still being computed.
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&bars->p_full[t][h]);
+                }
             }
             if (!ok) break;
             {

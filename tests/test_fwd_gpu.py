@@ -5,10 +5,12 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from io_aware_exact_31_b200 import binding
-from io_aware_exact_31_b200.workloads import WORKLOADS
+from io_aware_exact_31_b200.workloads import WORKLOADS, bf16_bits
 
-from _parity import check_forward_full, check_forward_sampled, gpu_forward, inputs
+from _parity import (TOL_GRAD_REL, TOL_LSE, TOL_O, check_forward_full, check_forward_sampled,
+                     fwd_errors, gpu_forward, grad_rel_err, inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +59,39 @@ def test_b4_h16_n2048_d64_causal_sampled():
     """The forward of the forward + backward workload, every CTA checked."""
     w = WORKLOADS["b4_h16_n2048_d64_causal_bwd"]
     check_forward_sampled(w.B, w.H, w.N, w.d, w.causal, n_random=4)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("p_drop", [0.0, 0.1])
+def test_late_dominant_key(d, causal, p_drop):
+    """One key in a late block (key 700 = 64 * ones) whose scores exceed the
+    earlier blocks' by up to ~2^250 for a quarter of the rows: the running
+    reference must move (rescale, or at d = 64 the redo of a block that
+    outgrows a reference taken without its row max) and O, LSE and the
+    gradients still match the oracle."""
+    B, H, N = 1, 2, 1024
+    x = inputs(B, H, N, d, seed=31, with_dO=True)
+    x["K"][:, :, 700, :] = 64.0
+    scale = 1.0 / math.sqrt(d)
+    q, k, v, do = (x[n].cuda() for n in ("Q", "K", "V", "dO"))
+    o, lse = binding.forward(q, k, v, causal=causal, scale=scale, dropout_p=p_drop, seed=5)
+    dq, dk, dv = binding.backward(q, k, v, o, do, lse, causal=causal, scale=scale,
+                                  dropout_p=p_drop, seed=5)
+    st, site = binding.check_device_error()
+    assert st == binding.FA_OK, f"device error {site:#x}"
+    bits = [bf16_bits(x[n]) for n in ("Q", "K", "V", "dO")]
+    if p_drop > 0:
+        O_ref, L_ref = oracle.attention_forward_dropout(*bits[:3], scale, causal, p_drop, 5, 0)
+        refs = oracle.attention_backward_dropout(*bits, scale, causal, p_drop, 5, 0)
+    else:
+        O_ref, L_ref = oracle.attention_forward(*bits[:3], scale, causal)
+        refs = oracle.attention_backward(*bits, scale, causal)
+    eo, el = fwd_errors(o, lse, O_ref, L_ref)
+    assert eo <= TOL_O and el <= TOL_LSE, f"max|dO|={eo:.3e} max|dLSE|={el:.3e}"
+    for name, g, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), refs):
+        e = grad_rel_err(g, r)
+        assert e <= TOL_GRAD_REL, f"{name}: {e:.3e}"
 
 
 def test_deterministic():
