@@ -40,9 +40,9 @@
 // threads issue the MMAs: warp 8 all S_t, warps 10 and 11 the P.V of tile 0
 // and tile 1, so that each issuing thread waits only on the barriers of its
 // own instructions.  The softmax waits for P.V_t(j-1)
-// (barrier pv_done) before it rescales O_t or overwrites P_t.  S_1(j) waits
-// until tile 0 is halfway through its exponentials of block j (barrier
-// exp_mark), which keeps the two tiles' exponential phases apart.
+// (barrier pv_done) before it rescales O_t or overwrites P_t.  One tile's S(j)
+// waits until the other tile is halfway through its exponentials of block j
+// (barrier exp_mark), which keeps the two tiles' exponential phases apart.
 #pragma once
 
 #include "philox.cuh"
@@ -110,7 +110,7 @@ struct FwdBars {
     uint64_t v_full[3], v_empty[3];
     uint64_t s_full[2], p_full[2][2], o_full[2];  // p_full[tile][key half]
     uint64_t s_free[2], pv_done[2];               // separate-P layout only
-    uint64_t exp_mark;                            // separate-P layout: tile 0 halfway through its exponentials
+    uint64_t exp_mark;                            // separate-P layout: the leading tile halfway through its exponentials
 };
 static_assert(sizeof(FwdBars) + 8 <= 256, "barrier area");
 
@@ -161,6 +161,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
         n_tile[t] = padding_cta ? 0 : p.causal ? min(last_row / FWD_BN + 1, n_kv) : n_kv;
     }
     const int n_blocks = n_tile[1];  // n_tile[0] <= n_tile[1] <= n_tile[0] + 1
+    // d = 64: the tile whose exponentials lead the other's by half a softmax
+    // (below).  With causal masking tile 1, which may have the extra block, so
+    // that the follower ends about when the leader does; otherwise tile 0
+    // (measured: 4x16x2048x64 causal 454 -> 476 TFLOP/s with tile 1 leading,
+    // 4x16x4096x64 704 -> 675).
+    const int lead = p.causal ? 1 : 0;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -325,21 +331,21 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     const int sk = j % C::NK;
                     if (!(ok = mbar_wait_warp(&bars->k_full[sk], (j / C::NK) & 1, g, 5))) break;
 #pragma unroll
-                    for (int t = 0; t < 2; ++t) {
+                    for (int tt = 0; tt < 2; ++tt) {
+                        const int t = (tt == 0) ? lead : 1 - lead;
                         if (j < n_tile[t]) {
                             if (j > 0 && !(ok = mbar_wait_warp(&bars->s_free[t], (j - 1) & 1, g, 15 + t)))
                                 break;
-                            // S_1(j) only once tile 0 has made the first half of
-                            // its weights of block j (barrier exp_mark, one
-                            // arrival per tile-0 warp).  Left alone the two tiles
-                            // run in lock step, both warps of a sub-partition
-                            // in their exponentials at once and then both idle
-                            // on the ex2 unit while they wait for S and load
-                            // it; held half a softmax apart every block, each
-                            // warp's loads and waits fall in the other's
-                            // exponentials.
-                            if (t == 1 && j < n_tile[0] &&
-                                !(ok = mbar_wait_warp(&bars->exp_mark, j & 1, g, 50)))
+                            // The follower's S(j) only once the leading tile has
+                            // made the first half of its weights of block j
+                            // (barrier exp_mark, one arrival per leading warp).
+                            // Left alone the two tiles run in lock step, both
+                            // warps of a sub-partition in their exponentials at
+                            // once and then both idle on the ex2 unit while they
+                            // wait for S and load it; held half a softmax apart
+                            // every block, each warp's loads and waits fall in
+                            // the other's exponentials.
+                            if (t != lead && !(ok = mbar_wait_warp(&bars->exp_mark, j & 1, g, 50)))
                                 break;
                             tc_fence_after();
                             issue_S(t, sk);
@@ -570,7 +576,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                 {
                     uint32_t pk[32];
                     exp_half(0, m_sub, pk);
-                    if (t == 0 && lane == 0) mbar_arrive(&bars->exp_mark);
+                    if (t == lead && lane == 0) mbar_arrive(&bars->exp_mark);
                     if (!(ok = mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, g, 23 + t))) break;
                     tc_fence_after();
                     store_P(0, pk);
@@ -611,7 +617,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ 
                     exp_half(h, m_sub, pk);
                     if constexpr (C::SEP) {
                         if (h == 0) {
-                            if (t == 0 && lane == 0) mbar_arrive(&bars->exp_mark);
+                            if (t == lead && lane == 0) mbar_arrive(&bars->exp_mark);
                             // P_t and O_t are free once P.V_t(j-1) has completed.
                             if (j > 0) {
                                 if (!(ok = mbar_wait_warp(&bars->pv_done[t], (j - 1) & 1, g, 23 + t)))
